@@ -1,0 +1,205 @@
+"""fp64 CPU oracle for the CSA lightning-indexer top-k step (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The product path (the CUDA library and its
+binding) never does, and the two share no code: the only thing both use is the
+seeded input generator in ``synth``.
+
+The arithmetic lives in ``oracle.c`` (plain loops, fp64, qsort); this module
+compiles it with gcc on first use and marshals numpy arrays to it.  The C
+file's header states the definition it follows ("StreamIndex: Memory-Bounded
+Compressed Sparse Attention via Streaming Top-k", Abstract) and the readings it
+takes where that text is silent.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc -O2, OpenMP, no fast-math, no
+    FMA contraction, so every fp64 operation rounds once as written)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I, L = ctypes.c_int, ctypes.c_int64
+        lib.oracle_visible.argtypes = [I, I, I]
+        lib.oracle_visible.restype = I
+        lib.oracle_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
+        lib.oracle_indexer_topk.restype = I
+        lib.oracle_indexer_topk_rows.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
+        lib.oracle_indexer_topk_rows.restype = I
+        lib.oracle_score_keys_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, I, P]
+        lib.oracle_score_keys_rows.restype = None
+        lib.oracle_row_absmax_rows.argtypes = [P, P, P, I, I, I, I, P, I, P]
+        lib.oracle_row_absmax_rows.restype = None
+        lib.oracle_topk_scores.argtypes = [P, I, I, I, I, I, P, I, P, P]
+        lib.oracle_topk_scores.restype = I
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_quantize_e4m3_rows.argtypes = [P, L, I, P, P]
+        lib.oracle_quantize_e4m3_rows.restype = None
+        lib.oracle_indexer_topk_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, P, P]
+        lib.oracle_indexer_topk_fp8_rows.restype = I
+        lib.oracle_score_keys_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, I, P]
+        lib.oracle_score_keys_fp8_rows.restype = None
+        _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: np.ndarray):
+    assert a.flags.c_contiguous
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def visible(t: int, T: int, m: int) -> int:
+    """Number of compressed keys visible to query t (keys j with (j+1)m-1 <= t)."""
+    return _load().oracle_visible(int(t), int(T), int(m))
+
+
+def indexer_topk(q, w, kc, m: int, k: int, rows=None):
+    """Oracle top-k from full tensors.
+
+    q [B,S,H,D] uint16 (bf16 bits), w [B,S,H] float32, kc [B,T,D] uint16.
+    rows: flat positions b*S+t to evaluate (default: all).
+    Returns (idx [n,k] int32, score [n,k] float64).
+    """
+    q, w, kc = _c(q, np.uint16), _c(w, np.float32), _c(kc, np.uint16)
+    B, S, H, D = q.shape
+    rows = _c(np.arange(B * S) if rows is None else rows, np.int64)
+    n = rows.size
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float64)
+    rc = _load().oracle_indexer_topk(_p(q), _p(w), _p(kc), B, S, H, D, m, k, _p(rows), n, _p(idx),
+                                     _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_indexer_topk: bad arguments")
+    return idx, sc
+
+
+def indexer_topk_rows(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
+    """Oracle top-k given only the listed queries' rows of q and w
+    (q_rows [n,H,D], w_rows [n,H]); rows are their flat positions b*S+t."""
+    q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
+    rows = _c(rows, np.int64)
+    n, H, D = q_rows.shape
+    B = kc.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float64)
+    rc = _load().oracle_indexer_topk_rows(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m, k,
+                                          _p(rows), n, _p(idx), _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_indexer_topk_rows: bad arguments")
+    return idx, sc
+
+
+def score_keys_rows(q_rows, w_rows, kc, S: int, m: int, rows, js):
+    """fp64 scores of keys js[i, :] (entries < 0 give nan) for the listed queries."""
+    q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
+    rows, js = _c(rows, np.int64), _c(js, np.int32)
+    n, H, D = q_rows.shape
+    out = np.full(js.shape, np.nan, dtype=np.float64)
+    _load().oracle_score_keys_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n, _p(js),
+                                   js.shape[1], _p(out))
+    return out
+
+
+def row_absmax_rows(q_rows, w_rows, kc, S: int, m: int, rows):
+    """max over visible keys of |score| for each listed query."""
+    q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
+    rows = _c(rows, np.int64)
+    n, H, D = q_rows.shape
+    out = np.empty(n, dtype=np.float64)
+    _load().oracle_row_absmax_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n,
+                                   _p(out))
+    return out
+
+
+def topk_scores(X, m: int, k: int, rows=None):
+    """Selection alone on given fp32 scores X [B,S,T].
+    Returns (idx [n,k] int32, score [n,k] float32 carrying the input bit patterns)."""
+    X = _c(X, np.float32)
+    B, S, T = X.shape
+    rows = _c(np.arange(B * S) if rows is None else rows, np.int64)
+    n = rows.size
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float32)
+    rc = _load().oracle_topk_scores(_p(X), B, S, T, m, k, _p(rows), n, _p(idx), _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_topk_scores: bad arguments")
+    return idx, sc
+
+
+def e4m3_decode(code: int) -> float:
+    return _load().oracle_e4m3_decode(int(code))
+
+
+def e4m3_encode(y: float) -> int:
+    return _load().oracle_e4m3_encode(float(y))
+
+
+def quantize_e4m3_rows(x):
+    """x [..., cols] uint16 bf16 bits -> (codes uint8 [..., cols], scale fp32 [...])."""
+    x = _c(x, np.uint16)
+    shp = x.shape
+    x2 = x.reshape(-1, shp[-1])
+    codes = np.empty(x2.shape, dtype=np.uint8)
+    scale = np.empty(x2.shape[0], dtype=np.float32)
+    _load().oracle_quantize_e4m3_rows(_p(x2), x2.shape[0], x2.shape[1], _p(codes), _p(scale))
+    return codes.reshape(shp), scale.reshape(shp[:-1])
+
+
+def indexer_topk_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, k: int, rows):
+    """Oracle top-k of the FP8 score (codes decoded exactly, scales applied in fp64).
+
+    q8_rows [n,H,D] uint8, sq_rows [n,H] fp32, w_rows [n,H] fp32 for the listed
+    queries; k8 [B,T,D] uint8, s_k [B,T] fp32."""
+    q8_rows, sq_rows, w_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32), _c(w_rows, np.float32)
+    k8, s_k, rows = _c(k8, np.uint8), _c(s_k, np.float32), _c(rows, np.int64)
+    n, H, D = q8_rows.shape
+    B = k8.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float64)
+    rc = _load().oracle_indexer_topk_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8),
+                                              _p(s_k), B, S, H, D, m, k, _p(rows), n, _p(idx),
+                                              _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_indexer_topk_fp8_rows: bad arguments")
+    return idx, sc
+
+
+def score_keys_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, rows, js):
+    q8_rows, sq_rows, w_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32), _c(w_rows, np.float32)
+    k8, s_k, rows, js = _c(k8, np.uint8), _c(s_k, np.float32), _c(rows, np.int64), _c(js, np.int32)
+    n, H, D = q8_rows.shape
+    out = np.full(js.shape, np.nan, dtype=np.float64)
+    _load().oracle_score_keys_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8), _p(s_k), S, H,
+                                       D, m, _p(rows), n, _p(js), js.shape[1], _p(out))
+    return out

@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA lightning-indexer top-k step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload v4flash_s16k] [--key-chunk C] [--fp8]
+
+A step is one pass of the whole hot path (score contraction on tensor cores,
+ReLU + weighted head sum, causal mask, streaming top-k and, when keys are
+chunked, the partition merge) over one batch of synthetic input.  The metric is
+causally visible query-key pairs per second; the JSON line also carries the
+achieved TFLOP/s against the measured bf16 tensor-core peak and the peak HBM.
+
+With N > 1 (one process per GPU under torch.distributed.run) every rank runs
+its own independent problem of the same shape (weak scaling, no data-path
+collective); the timed region is bracketed by barriers and its maximum over
+ranks is reported.  ``--impl reference`` times the fp64 CPU oracle instead
+(rank 0 only), on bounded samples of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "indexer query-key pairs/sec, TFLOPS vs B200 peak, peak HBM GB at 1 GPU"
+UNIT = "pairs/s"
+KERNEL_SRC = os.path.join(ROOT, "streaming_top_lightning_b200", "csrc", "k_score_topk.cu")
+
+
+def causal_pairs(S: int, T: int, m: int) -> int:
+    t = np.arange(S, dtype=np.int64)
+    return int(np.minimum(T, (t + 1) // m).sum())
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("k_score_topk.cu", "si_select.cuh", "si_common.cuh", "si_kernels.h"):
+        with open(os.path.join(ROOT, "streaming_top_lightning_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(workload: str, fp8: bool):
+    """DRAM bytes per launch of the score kernel from a committed ncu summary,
+    or None when absent or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    key = f"{workload}{'_fp8' if fp8 else ''}"
+    rec = d.get(key)
+    if not rec or rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "50"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+
+class OracleSample:
+    """A fixed set of query rows of the workload for timing the fp64 oracle,
+    sized (once, untimed) so that one call takes about ``budget_s``."""
+
+    def __init__(self, sh, budget_s: float, seed: int = 0):
+        import oracle
+
+        self.oracle, self.sh = oracle, sh
+        self.kc = synth.gen_kc(sh, seed)
+        S = sh.S
+        n = 2
+        while True:
+            self._set_rows(np.unique(np.linspace(S // 2, S - 1, n).astype(np.int64)), seed)
+            dt = self.run()
+            if dt >= budget_s * 0.5 or n >= S // 2:
+                break
+            n = int(min(S // 2, max(n * 2, n * budget_s / max(dt, 1e-3))))
+        self.desc = (f"{self.rows.size} query rows evenly spaced over t in [{S // 2}, {S - 1}] "
+                     f"of {sh.name} ({self.pairs} causal pairs), every visible key scored in "
+                     f"fp64, then sorted")
+
+    def _set_rows(self, rows, seed):
+        self.rows = rows
+        self.qr, self.wr = synth.gen_rows(self.sh, rows, seed)
+        self.pairs = int(np.minimum(self.sh.T, (rows % self.sh.S + 1) // self.sh.m).sum())
+
+    def run(self) -> float:
+        t0 = time.perf_counter()
+        self.oracle.indexer_topk_rows(self.qr, self.wr, self.kc, self.sh.S, self.sh.m,
+                                      self.sh.topk, self.rows)
+        return time.perf_counter() - t0
+
+
+def run_reference(args, sh):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = max(0.2, 120.0 / max(1, args.steps + args.warmup))
+    smp = OracleSample(sh, per_step)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = smp.run()
+        if i >= args.warmup:
+            times.append(dt)
+    value = smp.pairs / float(statistics.median(times))
+    P = causal_pairs(sh.S, sh.T, sh.m)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * P / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(sh, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": smp.oracle.threads(),
+                         "kind": "oracle", "sample": smp.desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(sh, args):
+    return {"workload": sh.name, "B": sh.B, "S": sh.S, "T": sh.T, "m": sh.m, "H_I": sh.H,
+            "d_I": sh.D, "topk": sh.topk, "key_chunk": args.key_chunk,
+            "score_path": "fp8-e4m3" if args.fp8 else "bf16",
+            "pairs_per_step": causal_pairs(sh.S, sh.T, sh.m),
+            "l2": "inputs larger than L2: q alone is "
+                  f"{sh.B * sh.S * sh.H * sh.D * (1 if args.fp8 else 2) / 1e6:.0f} MB per step",
+            "parallelism": f"replicas x{args.gpus} (independent problems)"}
+
+
+# --------------------------------------------------------------------------- native
+
+
+def run_native(args, sh):
+    import torch
+    import torch.distributed as dist
+
+    import streaming_top_lightning_b200 as stl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    seed = rank
+    P = causal_pairs(sh.S, sh.T, sh.m)
+    flops_per_pair = 2 * sh.H * sh.D
+    # inputs (host, pinned) generated blockwise; device copies
+    q_h = torch.empty((sh.B, sh.S, sh.H, sh.D), dtype=torch.int16).pin_memory()
+    synth.gen_q(sh, seed, out=q_h.numpy().view(np.uint16), threads=16)
+    w_h = torch.from_numpy(synth.gen_w(sh, seed)).pin_memory()
+    kc_h = torch.from_numpy(synth.gen_kc(sh, seed).view(np.int16)).pin_memory()
+    torch.cuda.synchronize()
+    free0, total = torch.cuda.mem_get_info()
+    torch.cuda.reset_peak_memory_stats()
+    q_d = q_h.to(dev).view(torch.bfloat16)
+    w_d = w_h.to(dev)
+    kc_d = kc_h.to(dev).view(torch.bfloat16)
+    opts = stl.options(key_chunk=args.key_chunk)
+    ws = torch.empty(max(16, stl.workspace_size(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, opts)),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32, device=dev)
+    score = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32, device=dev)
+    if args.fp8:
+        q8, s_q = stl.quantize_fp8_rows(q_d)
+        k8, s_k = stl.quantize_fp8_rows(kc_d)
+        del q_d
+        q_d = None
+
+        def step():
+            stl.indexer_topk_fp8(q8, s_q, w_d, k8, s_k, sh.m, sh.topk, out=(idx, score),
+                                 opts=opts, workspace=ws)
+    else:
+        def step():
+            stl.indexer_topk(q_d, w_d, kc_d, sh.m, sh.topk, out=(idx, score), opts=opts,
+                             workspace=ws)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    rc = stl.device_error()
+    if rc != 0:
+        raise RuntimeError(f"device error {rc} during warm-up")
+    peak_alloc = torch.cuda.max_memory_allocated()
+    free1, _ = torch.cuda.mem_get_info()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    rc = stl.device_error()
+    if rc != 0:
+        raise RuntimeError(f"device error {rc} in the timed region")
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    # end to end through the public API: host -> device inputs, the call,
+    # device -> host result, every step
+    idx_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32).pin_memory()
+    score_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32).pin_memory()
+    qe = torch.empty_like(q_h, device=dev)
+    we = torch.empty_like(w_h, device=dev)
+    ke = torch.empty_like(kc_h, device=dev)
+    h2d = q_h.numel() * 2 + w_h.numel() * 4 + kc_h.numel() * 2
+    d2h = idx_h.numel() * 4 + score_h.numel() * 4
+
+    def e2e_step():
+        qe.copy_(q_h, non_blocking=True)
+        we.copy_(w_h, non_blocking=True)
+        ke.copy_(kc_h, non_blocking=True)
+        if args.fp8:
+            a8, sa = stl.quantize_fp8_rows(qe.view(torch.bfloat16))
+            b8, sb = stl.quantize_fp8_rows(ke.view(torch.bfloat16))
+            stl.indexer_topk_fp8(a8, sa, we, b8, sb, sh.m, sh.topk, out=(idx, score), opts=opts,
+                                 workspace=ws)
+        else:
+            stl.indexer_topk(qe.view(torch.bfloat16), we, ke.view(torch.bfloat16), sh.m, sh.topk,
+                             out=(idx, score), opts=opts, workspace=ws)
+        idx_h.copy_(idx, non_blocking=True)
+        score_h.copy_(score, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    Ke = max(3, min(K, 20))
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    assert stl.device_error() == 0
+
+    ms_per_step = total_ms / K
+    value = world * P * sh.B / (ms_per_step / 1e3)
+    peaks, peak_src = measured_peaks()
+    flops_launch = flops_per_pair * P * sh.B
+    achieved = flops_launch / (launch_ms / 1e3) / 1e12
+    peak_tf = float(peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
+    tflops_step = flops_launch / (ms_per_step / 1e3) / 1e12
+    traffic = traffic_record(sh.name, args.fp8)
+    launches_per_step = 1 + (1 if args.key_chunk and args.key_chunk < sh.T else 0)
+    if args.fp8:
+        launches_per_step += 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3" if args.fp8 else "bf16",
+        "data": "synthetic (seeded; distributions of the workload recipe)",
+        "config": config_of(sh, args),
+        "tflops": tflops_step,
+        "tflops_frac_of_measured_peak": tflops_step / peak_tf,
+        "peak_hbm_gb": peak_alloc / 1e9,
+        "peak_hbm_gib": peak_alloc / 2 ** 30,
+        "hbm_in_use_delta_gb": (free0 - free1) / 1e9,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                     "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": traffic,
+                     "kernel": "k_score_topk", "peak_source": f"{peak_src} bf16_tflops (burst)"
+                     + (" x2 nominal fp8/bf16 ratio" if args.fp8 else ""),
+                     "algorithmic_flops_per_launch": flops_launch,
+                     "avg_launch_ms": launch_ms},
+        "e2e": {"value": world * P * sh.B * Ke / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        smp = OracleSample(sh, args.cpu_seconds)
+        secs = smp.run()
+        line["cpu_baseline"] = {"value": smp.pairs / secs, "unit": UNIT,
+                                "cores": smp.oracle.threads(), "kind": "oracle",
+                                "sample": smp.desc, "seconds": secs}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="v4flash_s16k", choices=sorted(synth.SHAPES))
+    ap.add_argument("--key-chunk", type=int, default=0)
+    ap.add_argument("--topk", type=int, default=0)
+    ap.add_argument("--fp8", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    sh = synth.shape(args.workload)
+    if args.topk:
+        sh = synth.shape(args.workload, topk=args.topk)
+    if args.impl == "reference":
+        return run_reference(args, sh)
+    return run_native(args, sh)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

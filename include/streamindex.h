@@ -1,0 +1,151 @@
+/*
+ * streamindex.h -- C ABI of the B200 (sm_100a) CSA lightning-indexer top-k library.
+ *
+ * The operation ("StreamIndex: Memory-Bounded Compressed Sparse Attention via
+ * Streaming Top-k", Abstract): in Compressed Sparse Attention a lightning
+ * indexer, a learned scoring projection over compressed keys, scores the keys
+ * each query can see and the top-k keys are kept per query; StreamIndex does
+ * this with a chunked partition-merge top-k driver that never materialises the
+ * [B,S,H_I,T] fp32 score tensor.  The abstract prints no formula; this library
+ * computes, for every batch b and query position t,
+ *
+ *     I[b,t,j] = sum_h w[b,t,h] * max(0, q[b,t,h,:] . kc[b,j,:])      (h < H_I)
+ *
+ * over the compressed keys j visible to t, i.e. (j+1)*m - 1 <= t, which is the
+ * first V_t = min(T, floor((t+1)/m)) keys (T = S/m, m the compression ratio,
+ * m = 4 for V4-Flash per the abstract).  It returns the min(topk, V_t) best
+ * keys per query, sorted by score descending with ties broken by the lower
+ * index (-0 and +0 are equal scores), followed by padding (index -1, score
+ * -inf).
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees them.  Layouts are dense row-major with the last named
+ *    dimension fastest.  bf16 is passed as 16-bit storage, E4M3 as bytes.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) unless stated otherwise.
+ *  - The return value is a status: SI_OK (0) or a negative SI_ERR_* code.
+ *    Argument errors are detected on the host before anything is launched.
+ *    After a non-zero status the outputs are undefined.
+ *  - Device-side waits are bounded; a kernel that gives up records a device
+ *    error word, read back by si_get_last_device_error().
+ *  - Limits: B >= 1; S >= 1 with S % m == 0; H_I in {8, 16, 32, 64};
+ *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I*d_I < 2^31 elements per
+ *    tensor row index; pointers 16-byte aligned.
+ */
+#ifndef STREAMINDEX_H
+#define STREAMINDEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------- */
+#define SI_OK 0
+#define SI_ERR_NULL -1           /* a required pointer is NULL */
+#define SI_ERR_DIM -2            /* a dimension is out of range (see limits above) */
+#define SI_ERR_TOPK -3           /* topk < 1 or topk > 2048 */
+#define SI_ERR_ALIGN -4          /* a pointer is not 16-byte aligned */
+#define SI_ERR_WORKSPACE -5      /* caller workspace too small */
+#define SI_ERR_CUDA -6           /* a CUDA runtime/driver call or launch failed */
+#define SI_ERR_DEVICE_TIMEOUT -7 /* a kernel gave up on a bounded wait */
+#define SI_ERR_OPTIONS -8        /* an si_options field is out of range */
+#define SI_ERR_UNSUPPORTED -9    /* no sm_100 device, or the device is not a B200-class part */
+
+#define SI_MAX_TOPK 2048
+
+/* Tuning and debug knobs.  Pass NULL for the defaults. */
+typedef struct si_options {
+  int key_chunk;        /* keys per chunk of the partition-merge driver, a
+                           multiple of 128; 0 = one chunk spans all keys of a
+                           query (no merge pass).  Default 0. */
+  int scratch_mb;       /* bound on partial-list scratch (MiB) used to size the
+                           query blocks of the chunked driver.  Default 512. */
+  int grid_ctas;        /* persistent CTAs; 0 = one per SM.  Default 0. */
+  int timeout_ms;       /* limit of any single device-side wait.  Default 2000. */
+  int debug_flags;      /* bit 0: the producer never issues its first load, so
+                           the first consumer wait must expire (tests the
+                           timeout path).  Default 0. */
+} si_options;
+
+/* ---- the indexer step ------------------------------------------------ */
+
+/*
+ * si_indexer_topk: score, mask and select in one pass (bf16 inputs).
+ *   q         bf16 [B,S,H_I,d_I]   indexer queries
+ *   w         fp32 [B,S,H_I]       per-head weights (signed)
+ *   kc        bf16 [B,T,d_I]       compressed keys, T = S/m
+ *   out_idx   int32 [B,S,topk]     selected key indices, -1 padding
+ *   out_score fp32  [B,S,topk]     their scores (fp32 accumulation), -inf padding
+ * Uses an internal workspace allocated with cudaMallocAsync on `stream` and
+ * released on the same stream before returning.
+ */
+int si_indexer_topk(const void* q, const float* w, const void* kc, int B, int S, int H_I, int d_I,
+                    int m, int topk, int32_t* out_idx, float* out_score, void* stream);
+
+/* Bytes of device workspace si_indexer_topk_ex needs for this problem. */
+int si_indexer_topk_workspace_size(int B, int S, int H_I, int d_I, int m, int topk,
+                                   const si_options* opt, size_t* bytes);
+
+/* As si_indexer_topk, with options and a caller-provided device workspace of
+ * ws_bytes (at least what si_indexer_topk_workspace_size reports). */
+int si_indexer_topk_ex(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                       int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                       const si_options* opt, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * si_indexer_topk_fp8: the same step with E4M3 operands and per-row scales.
+ *   q8  e4m3 [B,S,H_I,d_I] with s_q fp32 [B,S,H_I];  k8 e4m3 [B,T,d_I] with
+ *   s_k fp32 [B,T]; the score is sum_h w * max(0, s_q*s_k*(q8 . k8)), the
+ *   codes decoded exactly and the dot product accumulated in fp32.
+ * Scales must be positive.  Workspace as in si_indexer_topk_ex (the size query
+ * is the same call).
+ */
+int si_indexer_topk_fp8(const void* q8, const float* s_q, const float* w, const void* k8,
+                        const float* s_k, int B, int S, int H_I, int d_I, int m, int topk,
+                        int32_t* out_idx, float* out_score, const si_options* opt,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * si_quantize_fp8_rows: per-row E4M3 quantisation of a bf16 matrix.
+ *   x [rows, cols] bf16 -> x8 [rows, cols] e4m3 and scale [rows] fp32, with
+ *   scale = max|x_row| / 448 (1 for an all-zero row) and
+ *   x8 = E4M3 round-to-nearest-even, saturating, of x / scale (fp32 division).
+ * (The reference list of the abstract cites "FP8 Formats for Deep Learning"
+ * for the format; the per-row scaling is this library's reading.)
+ * cols must be a multiple of 8 and at most 4096.
+ */
+int si_quantize_fp8_rows(const void* x, int64_t rows, int cols, void* x8, float* scale,
+                         void* stream);
+
+/*
+ * si_topk_scores: the selection stage alone on a given fp32 score tensor.
+ *   scores [B,S,T] fp32; keys j >= V_t are ignored (never read).
+ *   Output as si_indexer_topk; selected scores keep their input bit patterns.
+ * Bit-exact: the same indices and bits as a plain sort of each row's visible
+ * scores under the order above.  Workspace: internal (cudaMallocAsync).
+ */
+int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, int32_t* out_idx,
+                   float* out_score, const si_options* opt, void* stream);
+
+/* ---- diagnostics ------------------------------------------------------ */
+
+/* Text for a status code (static storage). */
+const char* si_status_string(int status);
+
+/* Synchronises `stream`, then returns SI_OK, SI_ERR_DEVICE_TIMEOUT if a kernel
+ * since the previous call gave up on a bounded wait, or SI_ERR_CUDA; clears
+ * the device error word of the current device. */
+int si_get_last_device_error(void* stream);
+
+/* Library version as an integer, major*10000 + minor*100 + patch. */
+int si_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STREAMINDEX_H */

@@ -44,12 +44,16 @@ def _load():
         lib = ctypes.CDLL(build())
         P = ctypes.c_void_p
         I, L = ctypes.c_int, ctypes.c_int64
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = I
         lib.oracle_visible.argtypes = [I, I, I]
         lib.oracle_visible.restype = I
         lib.oracle_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
         lib.oracle_indexer_topk.restype = I
         lib.oracle_indexer_topk_rows.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
         lib.oracle_indexer_topk_rows.restype = I
+        lib.oracle_indexer_topk_rows_absmax.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P, P]
+        lib.oracle_indexer_topk_rows_absmax.restype = I
         lib.oracle_score_keys_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, I, P]
         lib.oracle_score_keys_rows.restype = None
         lib.oracle_row_absmax_rows.argtypes = [P, P, P, I, I, I, I, P, I, P]
@@ -77,6 +81,11 @@ def _c(a, dtype):
 def _p(a: np.ndarray):
     assert a.flags.c_contiguous
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def threads() -> int:
+    """OpenMP threads the oracle's row loops use."""
+    return _load().oracle_threads()
 
 
 def visible(t: int, T: int, m: int) -> int:
@@ -118,6 +127,22 @@ def indexer_topk_rows(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
     if rc != 0:
         raise ValueError("oracle_indexer_topk_rows: bad arguments")
     return idx, sc
+
+
+def indexer_topk_rows_absmax(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
+    """``indexer_topk_rows`` plus each row's max |score| over its visible keys."""
+    q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
+    rows = _c(rows, np.int64)
+    n, H, D = q_rows.shape
+    B = kc.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float64)
+    amax = np.empty(n, dtype=np.float64)
+    rc = _load().oracle_indexer_topk_rows_absmax(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m, k,
+                                                 _p(rows), n, _p(idx), _p(sc), _p(amax))
+    if rc != 0:
+        raise ValueError("oracle_indexer_topk_rows_absmax: bad arguments")
+    return idx, sc, amax
 
 
 def score_keys_rows(q_rows, w_rows, kc, S: int, m: int, rows, js):

@@ -31,6 +31,9 @@
  * with the codes decoded exactly to fp64.
  */
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -67,6 +70,15 @@ static double bf16_to_f64(uint16_t h) {
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* Threads the oracle's parallel loops use (1 without OpenMP). */
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /* Number of compressed keys query t can see: all j with (j+1)*m - 1 <= t. */
@@ -130,6 +142,42 @@ int oracle_indexer_topk_rows(const uint16_t* q_rows, const float* w_rows, const 
         oracle_topk_row(q_rows + (int64_t)i * H * D, w_rows + (int64_t)i * H,
                         kc + b * T * (int64_t)D, T, H, D, m, t, k, out_idx + (int64_t)i * k,
                         out_score + (int64_t)i * k);
+    }
+    return 0;
+}
+
+/* As oracle_indexer_topk_rows, also returning each row's largest |score|
+ * over its visible keys (out_absmax [n]); one scoring pass per row. */
+int oracle_indexer_topk_rows_absmax(const uint16_t* q_rows, const float* w_rows,
+                                    const uint16_t* kc, int B, int S, int H, int D, int m, int k,
+                                    const int64_t* rows, int n, int32_t* out_idx,
+                                    double* out_score, double* out_absmax) {
+    if (B < 1 || S < 1 || H < 1 || D < 1 || m < 1 || k < 1 || S % m != 0) return -1;
+    int T = S / m;
+    for (int i = 0; i < n; i++)
+        if (rows[i] < 0 || rows[i] >= (int64_t)B * S) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n; i++) {
+        int64_t b = rows[i] / S;
+        int t = (int)(rows[i] % S);
+        int V = oracle_visible(t, T, m);
+        const uint16_t* qr = q_rows + (int64_t)i * H * D;
+        const float* wr = w_rows + (int64_t)i * H;
+        const uint16_t* kcb = kc + b * T * (int64_t)D;
+        pair_t* p = (pair_t*)malloc(sizeof(pair_t) * (size_t)(V > 0 ? V : 1));
+        double mx = 0.0;
+        for (int j = 0; j < V; j++) {
+            p[j].s = oracle_score_row(qr, wr, kcb, H, D, j);
+            p[j].j = j;
+            if (fabs(p[j].s) > mx) mx = fabs(p[j].s);
+        }
+        qsort(p, (size_t)V, sizeof(pair_t), cmp_pair);
+        for (int r = 0; r < k; r++) {
+            out_idx[(int64_t)i * k + r] = r < V ? p[r].j : -1;
+            out_score[(int64_t)i * k + r] = r < V ? p[r].s : -INFINITY;
+        }
+        out_absmax[i] = mx;
+        free(p);
     }
     return 0;
 }

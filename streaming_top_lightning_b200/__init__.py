@@ -1,0 +1,166 @@
+"""B200 (sm_100a) CSA lightning-indexer top-k.
+
+Python face of libstreamindex.so.  It marshals torch CUDA tensors (device
+pointers, the current stream) into the C ABI of include/streamindex.h; every
+step of the computation runs in the library's CUDA kernels.  There is no CPU
+path: the calls raise if the library is not built or no sm_100 GPU is present.
+
+    idx, score = indexer_topk(q, w, kc, m=4, topk=512)
+
+q [B,S,H_I,d_I] bf16, w [B,S,H_I] fp32, kc [B,S/m,d_I] bf16, all on one CUDA
+device.  idx [B,S,topk] int32 (-1 padding), score [B,S,topk] fp32 (-inf padding).
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import SiOptions, StreamIndexError  # noqa: F401
+
+__all__ = [
+    "indexer_topk", "indexer_topk_fp8", "quantize_fp8_rows", "topk_scores", "workspace_size",
+    "device_error", "options", "version", "StreamIndexError",
+]
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, ndim, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def options(key_chunk: int = 0, scratch_mb: int = 0, grid_ctas: int = 0, timeout_ms: int = 0,
+            debug_flags: int = 0) -> SiOptions:
+    return SiOptions(key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags)
+
+
+def version() -> int:
+    return _lib.load().si_version()
+
+
+def workspace_size(B: int, S: int, H: int, D: int, m: int, topk: int, opts: SiOptions | None = None) -> int:
+    n = ctypes.c_size_t(0)
+    lib = _lib.load()
+    _lib.check("si_indexer_topk_workspace_size",
+               lib.si_indexer_topk_workspace_size(B, S, H, D, m, topk,
+                                                  ctypes.byref(opts) if opts else None,
+                                                  ctypes.byref(n)))
+    return n.value
+
+
+def _outputs(B, S, topk, device, out):
+    torch = _torch()
+    if out is not None:
+        idx, score = out
+        _need(idx, torch.int32, 3, "out_idx")
+        _need(score, torch.float32, 3, "out_score")
+        if tuple(idx.shape) != (B, S, topk) or tuple(score.shape) != (B, S, topk):
+            raise ValueError("out tensors must be [B,S,topk]")
+        return idx, score
+    return (torch.empty((B, S, topk), dtype=torch.int32, device=device),
+            torch.empty((B, S, topk), dtype=torch.float32, device=device))
+
+
+def indexer_topk(q, w, kc, m: int, topk: int, *, out=None, opts: SiOptions | None = None,
+                 workspace=None, stream=None):
+    """Top-k compressed keys per query (bf16 score path).  Returns (idx, score)."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    _need(w, torch.float32, 3, "w")
+    _need(kc, torch.bfloat16, 3, "kc")
+    B, S, H, D = q.shape
+    idx, score = _outputs(B, S, topk, q.device, out)
+    lib = _lib.load()
+    st = _stream(stream)
+    if opts is None and workspace is None:
+        rc = lib.si_indexer_topk(_ptr(q), _ptr(w), _ptr(kc), B, S, H, D, m, topk, _ptr(idx),
+                                 _ptr(score), st)
+        _lib.check("si_indexer_topk", rc)
+        return idx, score
+    need = workspace_size(B, S, H, D, m, topk, opts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = lib.si_indexer_topk_ex(_ptr(q), _ptr(w), _ptr(kc), B, S, H, D, m, topk, _ptr(idx),
+                                _ptr(score), ctypes.byref(opts) if opts else None,
+                                _ptr(workspace), workspace.numel(), st)
+    _lib.check("si_indexer_topk_ex", rc)
+    return idx, score
+
+
+def indexer_topk_fp8(q8, s_q, w, k8, s_k, m: int, topk: int, *, out=None,
+                     opts: SiOptions | None = None, workspace=None, stream=None):
+    """FP8 (E4M3) score path: q8 [B,S,H,D] and k8 [B,T,D] uint8 codes with
+    per-row scales s_q [B,S,H], s_k [B,T].  Returns (idx, score)."""
+    torch = _torch()
+    _need(q8, torch.uint8, 4, "q8")
+    _need(s_q, torch.float32, 3, "s_q")
+    _need(w, torch.float32, 3, "w")
+    _need(k8, torch.uint8, 3, "k8")
+    _need(s_k, torch.float32, 2, "s_k")
+    B, S, H, D = q8.shape
+    idx, score = _outputs(B, S, topk, q8.device, out)
+    need = workspace_size(B, S, H, D, m, topk, opts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q8.device)
+    lib = _lib.load()
+    rc = lib.si_indexer_topk_fp8(_ptr(q8), _ptr(s_q), _ptr(w), _ptr(k8), _ptr(s_k), B, S, H, D, m,
+                                 topk, _ptr(idx), _ptr(score),
+                                 ctypes.byref(opts) if opts else None, _ptr(workspace),
+                                 workspace.numel(), _stream(stream))
+    _lib.check("si_indexer_topk_fp8", rc)
+    return idx, score
+
+
+def quantize_fp8_rows(x, stream=None):
+    """Per-row E4M3 quantisation of a bf16 tensor [..., cols]: returns
+    (codes uint8 [..., cols], scale fp32 [...])."""
+    torch = _torch()
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 CUDA tensor")
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    rc = _lib.load().si_quantize_fp8_rows(_ptr(x), rows, cols, _ptr(x8), _ptr(scale),
+                                          _stream(stream))
+    _lib.check("si_quantize_fp8_rows", rc)
+    return x8, scale
+
+
+def topk_scores(scores, m: int, topk: int, *, out=None, opts: SiOptions | None = None,
+                stream=None):
+    """Selection alone on given fp32 scores [B,S,T] (causal rule with ratio m)."""
+    torch = _torch()
+    _need(scores, torch.float32, 3, "scores")
+    B, S, T = scores.shape
+    idx, score = _outputs(B, S, topk, scores.device, out)
+    rc = _lib.load().si_topk_scores(_ptr(scores), B, S, T, m, topk, _ptr(idx), _ptr(score),
+                                    ctypes.byref(opts) if opts else None, _stream(stream))
+    _lib.check("si_topk_scores", rc)
+    return idx, score
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and return the device status word as an SI status code."""
+    return _lib.load().si_get_last_device_error(_stream(stream))

@@ -1,0 +1,420 @@
+// The C ABI (include/streamindex.h): argument checks, workspace plan, tensor
+// maps and the chunked partition-merge driver loop.
+//
+// Driver ("StreamIndex: Memory-Bounded Compressed Sparse Attention via
+// Streaming Top-k", Abstract: a chunked partition-merge top-k driver that never
+// materialises the full score tensor).  Keys are split into chunks of
+// key_chunk keys; each (query tile, key chunk) unit leaves a sorted partial
+// list; the merge kernel folds them.  To keep the scratch bounded
+// independently of S, query tiles are processed in blocks sized so that one
+// block's partial lists fit the scratch budget: one score launch and one merge
+// launch per block.  With key_chunk = 0 a single chunk covers each query's
+// keys, units write the final answer directly and no merge pass runs.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "streamindex.h"
+#include "si_kernels.h"
+
+namespace si {
+
+__device__ uint32_t g_err_word;
+
+namespace {
+
+struct DevInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+  int max_smem = 0;
+  uint32_t* err = nullptr;
+};
+
+std::mutex g_mu;
+DevInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int dev_info(DevInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SI_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return SI_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return SI_ERR_CUDA;
+    d.err = static_cast<uint32_t*>(p);
+    d.ok = (major == 10 && minor == 0);
+    d.init = true;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return SI_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (!d.ok) return SI_ERR_UNSUPPORTED;
+  *out = &d;
+  return SI_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// 2-D row-major [rows, cols] tensor map with a {box_inner, box_rows} box and
+// the given swizzle; out-of-range rows read as zero.
+int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t rows,
+             uint64_t cols, uint32_t esz, uint32_t box_inner, uint32_t box_rows,
+             CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esz};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SI_OK : SI_ERR_CUDA;
+}
+
+struct Opts {
+  int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags;
+};
+
+int read_opts(const si_options* o, Opts* out) {
+  Opts d{0, 512, 0, 2000, 0};
+  if (o) {
+    d.key_chunk = o->key_chunk;
+    d.scratch_mb = o->scratch_mb > 0 ? o->scratch_mb : 512;
+    d.grid_ctas = o->grid_ctas;
+    d.timeout_ms = o->timeout_ms > 0 ? o->timeout_ms : 2000;
+    d.debug_flags = o->debug_flags;
+  }
+  if (d.key_chunk < 0 || (d.key_chunk % 128) != 0 || d.grid_ctas < 0 || d.scratch_mb > (1 << 20))
+    return SI_ERR_OPTIONS;
+  *out = d;
+  return SI_OK;
+}
+
+// The plan of one problem: tiles, chunks and query blocks.
+struct Plan {
+  int QT, G, T, C, nch_max, tb, n_blocks;
+  size_t counters_bytes, partial_bytes;
+  size_t ws_bytes() const { return align256(counters_bytes) + partial_bytes; }
+};
+
+Plan make_plan(int B, int S, int m, int K, int QT, const Opts& o) {
+  Plan p{};
+  p.QT = QT;
+  p.T = S / m;
+  p.G = (S + QT - 1) / QT;
+  const int tround = ((p.T > 0 ? p.T : 1) + 127) / 128 * 128;
+  p.C = o.key_chunk > 0 ? o.key_chunk : tround;
+  p.nch_max = p.T > 0 ? (p.T + p.C - 1) / p.C : 1;
+  if (p.nch_max <= 1) {
+    p.nch_max = 1;
+    p.tb = p.G;
+    p.partial_bytes = 0;
+  } else {
+    const size_t per_tile = (size_t)B * p.nch_max * QT * K * sizeof(uint64_t);
+    const size_t budget = (size_t)o.scratch_mb << 20;
+    size_t tb = budget / per_tile;
+    if (tb < 1) tb = 1;
+    if (tb > (size_t)p.G) tb = p.G;
+    p.tb = (int)tb;
+    p.partial_bytes = per_tile * p.tb;
+  }
+  p.n_blocks = (p.G + p.tb - 1) / p.tb;
+  p.counters_bytes = sizeof(int);  // one unit counter shared by every launch
+  return p;
+}
+
+int check_common(int B, int S, int m, int topk) {
+  if (B < 1 || S < 1 || m < 1 || S % m != 0) return SI_ERR_DIM;
+  if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
+  return SI_OK;
+}
+
+int check_indexer(const void* q, const void* w, const void* kc, int B, int S, int H, int D, int m,
+                  int topk, const void* oi, const void* os) {
+  if (!q || !w || !kc || !oi || !os) return SI_ERR_NULL;
+  int rc = check_common(B, S, m, topk);
+  if (rc) return rc;
+  if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
+  if ((int64_t)B * S * H >= ((int64_t)1 << 31)) return SI_ERR_DIM;
+  if (!aligned16(q) || !aligned16(w) || !aligned16(kc) || !aligned16(oi) || !aligned16(os))
+    return SI_ERR_ALIGN;
+  return SI_OK;
+}
+
+int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const void* kc,
+                const float* s_k, int B, int S, int H, int D, int m, int K, int32_t* out_idx,
+                float* out_score, const si_options* opt, void* ws, size_t ws_bytes,
+                cudaStream_t stream) {
+  int rc = check_indexer(q, w, kc, B, S, H, D, m, K, out_idx, out_score);
+  if (rc) return rc;
+  if (fp8 && (!s_q || !s_k)) return SI_ERR_NULL;
+  Opts o;
+  if ((rc = read_opts(opt, &o))) return rc;
+  DevInfo* dev;
+  if ((rc = dev_info(&dev))) return rc;
+  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem);
+  if (!sp_plan.ok) return SI_ERR_DIM;
+  const Plan pl = make_plan(B, S, m, K, sp_plan.QT, o);
+  if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
+  if (!aligned16(ws)) return SI_ERR_ALIGN;
+
+  int* counters = static_cast<int*>(ws);
+  uint64_t* partial =
+      pl.partial_bytes ? reinterpret_cast<uint64_t*>(static_cast<char*>(ws) +
+                                                     align256(pl.counters_bytes))
+                       : nullptr;
+  if (cudaMemsetAsync(counters, 0, pl.counters_bytes, stream) != cudaSuccess) return SI_ERR_CUDA;
+
+  const int esz = fp8 ? 1 : 2;
+  const int row_bytes = D * esz;
+  const int sw_bytes = row_bytes >= 128 ? 128 : row_bytes;
+  const CUtensorMapSwizzle sw =
+      sw_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapDataType dt =
+      fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap tm_q, tm_kc;
+  const int T = pl.T;
+  if ((rc = make_map(&tm_q, q, dt, (uint64_t)B * S * H, D, esz, sw_bytes / esz, 256, sw)))
+    return rc;
+  if ((rc = make_map(&tm_kc, kc, dt, (uint64_t)B * (T > 0 ? T : 1), D, esz, sw_bytes / esz, 128,
+                     sw)))
+    return rc;
+
+  // Every CTA takes units until one decode fails, so a launch advances the
+  // shared counter by exactly (its units + its grid).
+  int id_base = 0;
+  for (int blk = 0; blk < pl.n_blocks; ++blk) {
+    const int g_lo = blk * pl.tb;
+    const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
+    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base};
+    ScoreParams p{};
+    p.sel = SelParams{B, S, T, m, K, pl.QT, sp_plan.CS, g_lo, n_tiles, pl.nch_max,
+                      out_idx, out_score, partial};
+    p.ug = ug;
+    p.w = w;
+    p.s_q = s_q;
+    p.s_k = s_k;
+    p.counter = counters;
+    p.err = dev->err;
+    p.timeout_ns = (uint64_t)o.timeout_ms * 1000000ull;
+    p.nst = sp_plan.nst;
+    p.debug_flags = o.debug_flags;
+    const int units = host_count_units(ug);
+    int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
+    if (grid > units) grid = units;
+    if (grid < 1) grid = 1;
+    if (launch_score_topk(fp8, D, H, tm_q, tm_kc, p, grid, sp_plan.smem, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
+    id_base += units + grid;
+    if (pl.nch_max > 1 && launch_merge(partial, p.sel, ug, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
+  }
+  return SI_OK;
+}
+
+int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_options* opt,
+                  size_t* bytes) {
+  int rc = check_common(B, S, m, K);
+  if (rc) return rc;
+  if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
+  Opts o;
+  if ((rc = read_opts(opt, &o))) return rc;
+  const int QT = 256 / H;
+  const Plan pl = make_plan(B, S, m, K, QT, o);
+  *bytes = pl.ws_bytes();
+  (void)fp8;
+  return SI_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ unit counting
+static int host_tile_vmax(const UnitGrid& u, int g) {
+  int t = g * u.QT + u.QT - 1;
+  if (t > u.S - 1) t = u.S - 1;
+  const int v = (t + 1) / u.m;
+  return v < u.T ? v : u.T;
+}
+
+int host_tile_chunks(const UnitGrid& u, int g) {
+  const int v = host_tile_vmax(u, g);
+  return v <= 0 ? 1 : (v + u.C - 1) / u.C;
+}
+
+int host_count_units(const UnitGrid& u) {
+  int64_t n = 0;
+  for (int g = u.g_lo; g < u.g_lo + u.n_tiles; ++g) n += host_tile_chunks(u, g);
+  n *= u.B;
+  return n > 0x7FFFFFFF ? 0x7FFFFFFF : (int)n;
+}
+
+}  // namespace si
+
+using namespace si;
+
+extern "C" {
+
+int si_version(void) { return 100; }
+
+const char* si_status_string(int s) {
+  switch (s) {
+    case SI_OK: return "ok";
+    case SI_ERR_NULL: return "a required pointer is NULL";
+    case SI_ERR_DIM: return "a dimension is out of range";
+    case SI_ERR_TOPK: return "topk out of range (1..2048)";
+    case SI_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case SI_ERR_WORKSPACE: return "workspace too small";
+    case SI_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case SI_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case SI_ERR_OPTIONS: return "an option is out of range";
+    case SI_ERR_UNSUPPORTED: return "no sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+int si_indexer_topk_workspace_size(int B, int S, int H_I, int d_I, int m, int topk,
+                                   const si_options* opt, size_t* bytes) {
+  if (!bytes) return SI_ERR_NULL;
+  return workspace_for(false, S, B, H_I, d_I, m, topk, opt, bytes);
+}
+
+int si_indexer_topk_ex(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                       int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                       const si_options* opt, void* workspace, size_t ws_bytes, void* stream) {
+  return run_indexer(false, q, nullptr, w, kc, nullptr, B, S, H_I, d_I, m, topk, out_idx,
+                     out_score, opt, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int si_indexer_topk(const void* q, const float* w, const void* kc, int B, int S, int H_I, int d_I,
+                    int m, int topk, int32_t* out_idx, float* out_score, void* stream) {
+  size_t bytes = 0;
+  int rc = si_indexer_topk_workspace_size(B, S, H_I, d_I, m, topk, nullptr, &bytes);
+  if (rc) return rc;
+  rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return SI_ERR_CUDA;
+  rc = si_indexer_topk_ex(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score, nullptr, ws,
+                          bytes, stream);
+  if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;
+  return rc;
+}
+
+int si_indexer_topk_fp8(const void* q8, const float* s_q, const float* w, const void* k8,
+                        const float* s_k, int B, int S, int H_I, int d_I, int m, int topk,
+                        int32_t* out_idx, float* out_score, const si_options* opt,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  return run_indexer(true, q8, s_q, w, k8, s_k, B, S, H_I, d_I, m, topk, out_idx, out_score, opt,
+                     workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int si_quantize_fp8_rows(const void* x, int64_t rows, int cols, void* x8, float* scale,
+                         void* stream) {
+  if (!x || !x8 || !scale) return SI_ERR_NULL;
+  if (rows < 0 || cols < 8 || cols > 4096 || cols % 8 != 0) return SI_ERR_DIM;
+  if (!aligned16(x) || !aligned16(x8) || !aligned16(scale)) return SI_ERR_ALIGN;
+  DevInfo* dev;
+  int rc = dev_info(&dev);
+  if (rc) return rc;
+  return launch_quantize_fp8(static_cast<const uint16_t*>(x), rows, cols,
+                             static_cast<uint8_t*>(x8), scale,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SI_OK
+             : SI_ERR_CUDA;
+}
+
+int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, int32_t* out_idx,
+                   float* out_score, const si_options* opt, void* stream) {
+  if (!scores || !out_idx || !out_score) return SI_ERR_NULL;
+  if (B < 1 || S < 1 || T < 1 || m < 1) return SI_ERR_DIM;
+  if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
+  if ((int64_t)B * S * T >= ((int64_t)1 << 40)) return SI_ERR_DIM;
+  if (!aligned16(scores) || !aligned16(out_idx) || !aligned16(out_score)) return SI_ERR_ALIGN;
+  Opts o;
+  int rc = read_opts(opt, &o);
+  if (rc) return rc;
+  DevInfo* dev;
+  if ((rc = dev_info(&dev))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int QT = 4, CS = 1024;
+  // the selection-only path sees T keys per row; m still sets visibility
+  Plan pl{};
+  {
+    pl.QT = QT;
+    pl.T = T;
+    pl.G = (S + QT - 1) / QT;
+    const int tround = (T + 127) / 128 * 128;
+    pl.C = o.key_chunk > 0 ? o.key_chunk : tround;
+    pl.nch_max = (T + pl.C - 1) / pl.C;
+    if (pl.nch_max <= 1) {
+      pl.nch_max = 1;
+      pl.tb = pl.G;
+      pl.partial_bytes = 0;
+    } else {
+      const size_t per_tile = (size_t)B * pl.nch_max * QT * topk * sizeof(uint64_t);
+      size_t tb = (((size_t)o.scratch_mb) << 20) / per_tile;
+      if (tb < 1) tb = 1;
+      if (tb > (size_t)pl.G) tb = pl.G;
+      pl.tb = (int)tb;
+      pl.partial_bytes = per_tile * pl.tb;
+    }
+    pl.n_blocks = (pl.G + pl.tb - 1) / pl.tb;
+    pl.counters_bytes = sizeof(int);
+  }
+  const size_t bytes = pl.ws_bytes();
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return SI_ERR_CUDA;
+  int* counters = static_cast<int*>(ws);
+  uint64_t* partial = pl.partial_bytes ? reinterpret_cast<uint64_t*>(
+                                             static_cast<char*>(ws) + align256(pl.counters_bytes))
+                                       : nullptr;
+  rc = SI_OK;
+  if (cudaMemsetAsync(counters, 0, pl.counters_bytes, st) != cudaSuccess) rc = SI_ERR_CUDA;
+  int id_base = 0;
+  for (int blk = 0; rc == SI_OK && blk < pl.n_blocks; ++blk) {
+    const int g_lo = blk * pl.tb;
+    const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
+    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base};
+    SelParams sp{B, S, T, m, topk, QT, CS, g_lo, n_tiles, pl.nch_max, out_idx, out_score, partial};
+    const int units = host_count_units(ug);
+    int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
+    if (grid > units) grid = units;
+    if (grid < 1) grid = 1;
+    if (launch_topk_scores(scores, sp, ug, counters, dev->err,
+                           (uint64_t)o.timeout_ms * 1000000ull, grid, st) != cudaSuccess)
+      rc = SI_ERR_CUDA;
+    else if (pl.nch_max > 1 && launch_merge(partial, sp, ug, st) != cudaSuccess)
+      rc = SI_ERR_CUDA;
+    id_base += units + grid;
+  }
+  if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;
+  return rc;
+}
+
+int si_get_last_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SI_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof v) != cudaSuccess) return SI_ERR_CUDA;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero) != cudaSuccess) return SI_ERR_CUDA;
+  if (v & SI_DEVERR_TIMEOUT) return SI_ERR_DEVICE_TIMEOUT;
+  return v ? SI_ERR_CUDA : SI_OK;
+}
+
+}  // extern "C"

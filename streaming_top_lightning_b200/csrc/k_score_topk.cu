@@ -1,0 +1,474 @@
+// Fused lightning-indexer score + streaming top-k on 5th-generation tensor cores.
+//
+// "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
+// Top-k", Abstract: a lightning indexer scores the compressed keys, the top-k
+// are selected per query, and the [B,S,H_I,T] fp32 score tensor is never
+// materialised.  Score read as I[t,j] = sum_h w[t,h] * max(0, q[t,h,:].kc[j,:]),
+// key j visible to t iff (j+1)*m - 1 <= t.
+//
+// Orientation: compressed keys on the MMA M dimension (128 TMEM lanes), the
+// QT = 256/H_I queries of a query tile times their H_I heads on N = 256.  So
+// D[j, (t,h)] = kc[j] . q[t,h] lands in TMEM with one key per lane, and each
+// epilogue thread reduces the heads of its own key without any cross-lane
+// traffic: one max and half a packed FMA per accumulator element.
+//
+// Warp roles (320 threads, one CTA per SM, persistent):
+//   warp 0     TMA producer and unit scheduler: takes (tile, chunk) units from
+//              a global counter, loads the query tile once per unit and streams
+//              128-key tiles of kc through an NST-stage mbarrier ring;
+//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma (one thread)
+//              into two 256-column accumulators used alternately;
+//   warps 2-5  epilogue: tcgen05.ld, ReLU, w-weighted head sum (x s_k for FP8),
+//              scores into a shared-memory strip; never to global memory;
+//   warps 6-9  streaming selection (si_select.cuh) on the strips.
+// Every wait is bounded (si_common.cuh); on expiry the CTA drains its own
+// asynchronous copies and MMAs, frees TMEM and exits with an error word set.
+#include "si_kernels.h"
+
+namespace si {
+
+constexpr int kThreads = 320;
+constexpr int kRing = 4;        // unit ring depth
+constexpr int kN = 256;         // MMA N: query-tile rows (QT * H)
+constexpr int kM = 128;         // MMA M: keys per tile
+constexpr int kEpiWarp0 = 2;    // first epilogue warp
+constexpr int kSelWarp0 = 6;    // first selection warp
+
+struct UnitInfo {
+  int valid, b, g, c, kbeg, kend, ntiles, direct;
+};
+
+struct ScoreCtlSmem {
+  uint64_t full[8], empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t q_full, q_empty;
+  uint64_t unit_full[kRing], unit_empty[kRing];
+  uint64_t strip_full[2], strip_empty[2];
+  uint64_t drain;
+  UnitInfo ring[kRing];
+  StripMeta meta[2];
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+template <bool FP8, int D>
+struct OperandGeom {
+  static constexpr int kEsz = FP8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kEsz;                      // bytes of one row
+  static constexpr int kSw = kRowBytes >= 128 ? 128 : kRowBytes;  // swizzle span
+  static constexpr int kKBlocks = kRowBytes / kSw;                // K-blocks per row
+  static constexpr int kKSteps = kRowBytes / 32;                  // MMA instructions per tile
+  static constexpr int kQBytes = kN * kRowBytes;
+  static constexpr int kKcBytes = kM * kRowBytes;
+};
+
+template <int SW>
+SI_DEV uint64_t sdesc(uint32_t saddr) {
+  // K-major, swizzled: 8-row groups SW*8 bytes apart.  Layout code: 128B -> 2,
+  // 64B -> 4 (see the descriptor field notes in si_common.cuh).
+  constexpr uint64_t kLayout = SW == 128 ? 2u : 4u;
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
+         ((uint64_t)((SW * 8) >> 4) << 32) | ((uint64_t)1u << 46) | (kLayout << 61);
+}
+
+SI_DEV void tmem_ld_fence(float (&v)[32]) {
+  asm volatile(""
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]),
+                 "+f"(v[6]), "+f"(v[7]), "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]),
+                 "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]), "+f"(v[16]), "+f"(v[17]),
+                 "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+                 "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]),
+                 "+f"(v[30]), "+f"(v[31]));
+}
+
+// Weighted ReLU head sum of one 32-column chunk into the per-query packed
+// accumulators.  Column c of the chunk is query (ch*32 + c) / H, head
+// (ch*32 + c) % H; w2 holds the unit's weights as float2 pairs.
+template <int H, int QT>
+SI_DEV void epi_chunk(int ch, const float (&v)[32], const float2* w2, float2 (&acc)[QT]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const int col = ch * 32 + e;
+    const int qi = col / H;
+    const float2 wv = w2[col >> 1];
+    const float2 r = make_float2(fmaxf(v[e], 0.0f), fmaxf(v[e + 1], 0.0f));
+    acc[qi] = __ffma2_rn(wv, r, acc[qi]);
+  }
+}
+
+template <bool FP8, int D, int H>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_score_topk(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                 const ScoreParams p) {
+  using G = OperandGeom<FP8, D>;
+  constexpr int QT = kN / H;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled operand tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const SelParams& sp = p.sel;
+  const int K = sp.K, CS = sp.CS, NST = p.nst;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  uint8_t* q_s = smem;
+  uint8_t* kc_s = q_s + G::kQBytes;
+  float* strip = reinterpret_cast<float*>(kc_s + (size_t)NST * G::kKcBytes);
+  uint64_t* lists = reinterpret_cast<uint64_t*>(strip + 2 * QT * CS);
+  uint64_t* cand = lists + (size_t)QT * K;
+  float* w_s = reinterpret_cast<float*>(cand + kSelWarps * kCandCap);  // [4 warps][kN]
+  ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + 4 * kN);
+
+  const uint32_t q_addr = smem_u32(q_s), kc_addr = smem_u32(kc_s);
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(smem_u32(&cs->full[s]), 1);
+      mbar_init(smem_u32(&cs->empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&cs->acc_full[i]), 1);
+      mbar_init(smem_u32(&cs->acc_empty[i]), 128);
+      mbar_init(smem_u32(&cs->strip_full[i]), 128);
+      mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);
+    }
+    mbar_init(smem_u32(&cs->q_full), 1);
+    mbar_init(smem_u32(&cs->q_empty), 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_u32(&cs->unit_full[i]), 1);
+      mbar_init(smem_u32(&cs->unit_empty[i]), 1 + 4);
+    }
+    mbar_init(smem_u32(&cs->drain), 1);
+    cs->abort = 0u;
+    mbar_fence_init();
+  }
+  for (int i = tid; i < QT * K; i += kThreads) lists[i] = 0ull;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&cs->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = cs->tmem_base;
+  Ctl ctl{p.err, &cs->abort, p.timeout_ns};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kc);
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_k = policy_evict_last();
+      uint32_t ring_it = 0, kstage = 0, q_it = 0;
+      bool q_issued = false;
+      bool skipped = false;  // debug: one key tile deliberately never loaded
+      int skipped_stage = -1;
+      for (;;) {
+        const int id = atomicAdd(p.counter, 1) - p.ug.id_base;
+        int b = 0, g = 0, c = 0;
+        const bool ok = unit_decode(p.ug, id, b, g, c);
+        const int r = ring_it % kRing;
+        if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl)) break;
+        UnitInfo u{0, 0, 0, 0, 0, 0, 0, 0};
+        if (ok) {
+          const int vmax = tile_vmax(p.ug, g);
+          u.valid = 1;
+          u.b = b;
+          u.g = g;
+          u.c = c;
+          u.kbeg = c * p.ug.C;
+          u.kend = min(u.kbeg + p.ug.C, vmax);
+          u.ntiles = u.kend > u.kbeg ? (u.kend - u.kbeg + kM - 1) / kM : 0;
+          u.direct = tile_chunks(p.ug, g) == 1;
+        }
+        cs->ring[r] = u;
+        mbar_arrive(smem_u32(&cs->unit_full[r]));
+        ++ring_it;
+        if (!ok) break;
+        if (u.ntiles == 0) continue;
+        // query tile: rows (b*S + g*QT)*H .. +256 of q viewed as [B*S*H, D]
+        if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl)) break;
+        const uint32_t qb = smem_u32(&cs->q_full);
+        mbar_arrive_expect_tx(qb, G::kQBytes);
+        const int qrow = (b * sp.S + g * QT) * H;
+#pragma unroll
+        for (int kb = 0; kb < G::kKBlocks; ++kb)
+          tma_load_2d(q_addr + kb * (kN * G::kSw), &tm_q, qb, kb * (G::kSw / G::kEsz), qrow, pol_q);
+        q_issued = true;
+        ++q_it;
+        // key tiles
+        bool stop = false;
+        for (int i = 0; i < u.ntiles; ++i) {
+          const int s = kstage % NST;
+          if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl)) {
+            stop = true;
+            break;
+          }
+          const uint32_t fb = smem_u32(&cs->full[s]);
+          mbar_arrive_expect_tx(fb, G::kKcBytes);
+          if ((p.debug_flags & 1) && !skipped) {
+            skipped = true;  // the consumer's wait on this stage must expire
+            skipped_stage = s;
+          } else {
+            const int krow = b * sp.T + u.kbeg + i * kM;
+            const uint32_t dst = kc_addr + s * G::kKcBytes;
+#pragma unroll
+            for (int kb = 0; kb < G::kKBlocks; ++kb)
+              tma_load_2d(dst + kb * (kM * G::kSw), &tm_kc, fb, kb * (G::kSw / G::kEsz), krow,
+                          pol_k);
+          }
+          ++kstage;
+        }
+        if (stop) break;
+      }
+      // drain: wait (bounded, regardless of abort) for every copy this thread
+      // issued to land before the CTA may exit
+      Ctl drain_ctl{p.err, nullptr, p.timeout_ns};
+      uint32_t dummy = 0;
+      drain_ctl.abort = &dummy;
+      for (uint32_t n = (kstage > (uint32_t)NST ? kstage - NST : 0); n < kstage; ++n) {
+        const int s = n % NST;
+        if (s == skipped_stage) continue;
+        mbar_wait(smem_u32(&cs->full[s]), (n / NST) & 1u, drain_ctl);
+      }
+      if (q_issued) mbar_wait(smem_u32(&cs->q_full), (q_it - 1) & 1u, drain_ctl);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = FP8 ? idesc_make(0, 0, kM, kN) : idesc_make(1, 1, kM, kN);
+      uint32_t ring_it = 0, kstage = 0, acc_it = 0, q_it = 0;
+      for (;;) {
+        const int r = ring_it % kRing;
+        if (!mbar_wait(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl)) break;
+        const UnitInfo u = cs->ring[r];  // ordered after the acquiring wait
+        mbar_arrive(smem_u32(&cs->unit_empty[r]));
+        ++ring_it;
+        if (!u.valid) break;
+        if (u.ntiles == 0) continue;
+        if (!mbar_wait(smem_u32(&cs->q_full), q_it & 1u, ctl)) break;
+        tc_fence_after();
+        bool stop = false;
+        for (int i = 0; i < u.ntiles; ++i) {
+          const int s = kstage % NST;
+          if (!mbar_wait(smem_u32(&cs->full[s]), (kstage / NST) & 1u, ctl)) {
+            stop = true;
+            break;
+          }
+          const int ab = acc_it & 1;
+          if (!mbar_wait(smem_u32(&cs->acc_empty[ab]), ((acc_it >> 1) & 1u) ^ 1u, ctl)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + ab * kN;
+          const uint32_t a0 = kc_addr + s * G::kKcBytes;
+#pragma unroll
+          for (int k = 0; k < G::kKSteps; ++k) {
+            constexpr int kPerBlock = G::kSw / 32;
+            const int kb = k / kPerBlock, kin = k % kPerBlock;
+            const uint64_t ad = sdesc<G::kSw>(a0 + kb * (kM * G::kSw) + kin * 32);
+            const uint64_t bd = sdesc<G::kSw>(q_addr + kb * (kN * G::kSw) + kin * 32);
+            if (FP8) umma_f8(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+            else umma_bf16(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&cs->empty[s]));
+          umma_commit(smem_u32(&cs->acc_full[ab]));
+          ++kstage;
+          ++acc_it;
+        }
+        if (stop) break;
+        umma_commit(smem_u32(&cs->q_empty));
+        ++q_it;
+      }
+      // drain: all MMAs issued by this thread complete before TMEM is freed
+      umma_commit(smem_u32(&cs->drain));
+      uint32_t dummy = 0;
+      Ctl drain_ctl{p.err, &dummy, p.timeout_ns};
+      mbar_wait(smem_u32(&cs->drain), 0u, drain_ctl);
+    }
+  } else if (warp < kSelWarp0) {
+    // ---------------------------------------------------------- epilogue
+    const int ew = warp - kEpiWarp0;  // 0..3
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int kl = quad * 32 + lane;  // key within the tile
+    float* wq = w_s + ew * kN;        // this warp's private copy of the unit's weights
+    const float2* w2 = reinterpret_cast<const float2*>(wq);
+    uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
+    for (;;) {
+      const int r = ring_it % kRing;
+      if (!mbar_wait_warp(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl)) break;
+      const UnitInfo u = cs->ring[r];  // ordered after the acquiring wait
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&cs->unit_empty[r]));
+      ++ring_it;
+      if (!u.valid) {
+        // no more work: pass the end marker to the selection warps
+        const int slot = strip_it & 1;
+        if (mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it >> 1) & 1u) ^ 1u, ctl)) {
+          if (ew == 0 && lane == 0) cs->meta[slot].valid = 0;
+          mbar_arrive(smem_u32(&cs->strip_full[slot]));
+        }
+        break;
+      }
+      // the unit's weights (FP8: folded with the query row scales, which are
+      // positive, so relu(s*x) = s*relu(x))
+      const int64_t wrow = (int64_t)u.b * sp.S + (int64_t)u.g * QT;
+      for (int i = lane; i < kN; i += 32) {
+        const int qi = i / H;
+        float wv = 0.0f;
+        if (u.g * QT + qi < sp.S) {
+          wv = p.w[wrow * H + i];
+          if (FP8) wv *= p.s_q[wrow * H + i];
+        }
+        wq[i] = wv;
+      }
+      __syncwarp();
+      int pos = 0, j_strip = u.kbeg;
+      bool stop = false;
+      for (int i = 0; i < u.ntiles || (i == 0 && u.ntiles == 0); ++i) {
+        const int slot = strip_it & 1;
+        if (pos == 0) {
+          if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it >> 1) & 1u) ^ 1u,
+                              ctl)) {
+            stop = true;
+            break;
+          }
+        }
+        if (u.ntiles > 0) {
+          const int ab = acc_it & 1;
+          if (!mbar_wait_warp(smem_u32(&cs->acc_full[ab]), (acc_it >> 1) & 1u, ctl)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ab * kN;
+          float2 acc[QT];
+#pragma unroll
+          for (int qi = 0; qi < QT; ++qi) acc[qi] = make_float2(0.0f, 0.0f);
+          float va[32], vb[32];
+          tmem_ld32(taddr, va);
+          tmem_ld_wait();
+          tmem_ld_fence(va);
+#pragma unroll
+          for (int ch = 0; ch < kN / 32; ch += 2) {
+            tmem_ld32(taddr + (ch + 1) * 32, vb);
+            epi_chunk<H, QT>(ch, va, w2, acc);
+            tmem_ld_wait();
+            tmem_ld_fence(vb);
+            if (ch + 2 < kN / 32) tmem_ld32(taddr + (ch + 2) * 32, va);
+            epi_chunk<H, QT>(ch + 1, vb, w2, acc);
+            if (ch + 2 < kN / 32) {
+              tmem_ld_wait();
+              tmem_ld_fence(va);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&cs->acc_empty[ab]));
+          ++acc_it;
+          float skj = 1.0f;
+          if (FP8) {
+            const int j = u.kbeg + i * kM + kl;
+            skj = j < sp.T ? p.s_k[(int64_t)u.b * sp.T + j] : 0.0f;
+          }
+          float* st = strip + (size_t)slot * QT * CS + pos + kl;
+#pragma unroll
+          for (int qi = 0; qi < QT; ++qi) {
+            float s = acc[qi].x + acc[qi].y;
+            if (FP8) s *= skj;
+            st[(size_t)qi * CS] = s;
+          }
+        }
+        pos += kM;
+        const bool last = (i + 1 >= u.ntiles);
+        if (pos >= CS || last) {
+          if (ew == 0 && lane == 0) {
+            const int nk = max(0, min(CS, u.kend - j_strip));
+            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0, u.direct};
+          }
+          mbar_arrive(smem_u32(&cs->strip_full[slot]));
+          ++strip_it;
+          pos = 0;
+          j_strip += CS;
+        }
+      }
+      if (stop) break;
+    }
+  } else {
+    // ---------------------------------------------------------- selection
+    SelSmem sm{lists, cand, strip, cs->meta, smem_u32(&cs->strip_full[0]),
+               smem_u32(&cs->strip_empty[0])};
+    select_loop(sp, sm, ctl, warp - kSelWarp0, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool FP8, int D, int H>
+static cudaError_t launch_t(const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
+                            const ScoreParams& p, int grid, size_t smem, cudaStream_t stream) {
+  auto kern = k_score_topk<FP8, D, H>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(tm_q, tm_kc, p);
+  return cudaGetLastError();
+}
+
+template <bool FP8, int D>
+static cudaError_t launch_h(int H, const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
+                            const ScoreParams& p, int grid, size_t smem, cudaStream_t stream) {
+  switch (H) {
+    case 8: return launch_t<FP8, D, 8>(tm_q, tm_kc, p, grid, smem, stream);
+    case 16: return launch_t<FP8, D, 16>(tm_q, tm_kc, p, grid, smem, stream);
+    case 32: return launch_t<FP8, D, 32>(tm_q, tm_kc, p, grid, smem, stream);
+    case 64: return launch_t<FP8, D, 64>(tm_q, tm_kc, p, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
+                              const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
+                              size_t smem, cudaStream_t stream) {
+  if (fp8) {
+    if (D == 128) return launch_h<true, 128>(H, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 64) return launch_h<true, 64>(H, tm_q, tm_kc, p, grid, smem, stream);
+  } else {
+    if (D == 128) return launch_h<false, 128>(H, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 64) return launch_h<false, 64>(H, tm_q, tm_kc, p, grid, smem, stream);
+  }
+  return cudaErrorInvalidValue;
+}
+
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
+  ScorePlan pl{};
+  const int esz = fp8 ? 1 : 2;
+  const int QT = kN / H;
+  const size_t q_bytes = (size_t)kN * D * esz;
+  const size_t kc_bytes = (size_t)kM * D * esz;
+  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(uint64_t) * QT * K +
+                       sizeof(uint64_t) * kSelWarps * kCandCap + sizeof(float) * 4 * kN +
+                       sizeof(ScoreCtlSmem);
+  pl.QT = QT;
+  pl.ok = false;
+  // prefer long strips, but keep at least 3 pipeline stages when possible
+  for (int min_st = 3; min_st >= 2 && !pl.ok; --min_st) {
+    for (int cs = 1024; cs >= kM; cs >>= 1) {
+      const size_t strip = sizeof(float) * 2 * QT * cs;
+      if (fixed + strip + min_st * kc_bytes > (size_t)max_smem) continue;
+      int nst = (int)((max_smem - fixed - strip) / kc_bytes);
+      if (nst > 6) nst = 6;
+      pl.CS = cs;
+      pl.nst = nst;
+      pl.smem = fixed + strip + nst * kc_bytes;
+      pl.ok = true;
+      break;
+    }
+  }
+  return pl;
+}
+
+}  // namespace si

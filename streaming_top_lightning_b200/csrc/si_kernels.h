@@ -1,0 +1,56 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "si_select.cuh"
+
+namespace si {
+
+// Parameters of the fused score + select kernel.
+struct ScoreParams {
+  SelParams sel;
+  UnitGrid ug;
+  const float* w;      // [B*S, H] fp32 head weights
+  const float* s_q;    // FP8 only: [B*S, H] query row scales
+  const float* s_k;    // FP8 only: [B*T] key row scales
+  int* counter;        // shared unit counter; this launch's ids start at ug.id_base
+  uint32_t* err;       // device error word
+  uint64_t timeout_ns; // limit of any single wait
+  int nst;             // key-tile pipeline stages
+  int debug_flags;     // bit 0: skip the first key-tile load (timeout test)
+};
+
+// Shared-memory plan of the fused kernel for one problem shape.
+struct ScorePlan {
+  int QT;        // queries per tile (256 / H)
+  int CS;        // keys per score strip
+  int nst;       // pipeline stages
+  size_t smem;   // dynamic shared memory bytes
+  bool ok;
+};
+
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem);
+
+cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
+                              const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
+                              size_t smem, cudaStream_t stream);
+
+size_t topk_scores_smem_bytes(int QT, int K, int CS);
+cudaError_t launch_topk_scores(const float* X, const SelParams& sp, const UnitGrid& ug,
+                               int* counter, uint32_t* err, uint64_t timeout_ns, int grid,
+                               cudaStream_t stream);
+
+cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
+                         cudaStream_t stream);
+
+cudaError_t launch_quantize_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* x8,
+                                float* scale, cudaStream_t stream);
+
+// Number of units (query tile x key chunk x batch) in a launch.
+int host_count_units(const UnitGrid& u);
+int host_tile_chunks(const UnitGrid& u, int g);
+
+}  // namespace si

@@ -1,0 +1,77 @@
+"""The C-ABI library: builds, loads, exports every symbol include/*.h declares,
+and rejects bad arguments on the host before any CUDA work."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from streaming_top_lightning_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(si_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations found"
+    assert declared == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert lib.si_status_string(0) == b"ok"
+    for code in range(-1, -10, -1):
+        assert lib.si_status_string(code) != b"unknown status"
+    assert lib.si_version() >= 100
+
+
+def _ws(lib, B, S, H, D, m, k, opts=None):
+    n = ctypes.c_size_t(0)
+    rc = lib.si_indexer_topk_workspace_size(B, S, H, D, m, k,
+                                            ctypes.byref(opts) if opts else None, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_and_validation(lib):
+    rc, n = _ws(lib, 1, 16384, 64, 128, 4, 512)
+    assert rc == 0 and n >= 4          # single chunk: just the unit counter
+    opts = _lib.SiOptions(1024, 64, 0, 0, 0)
+    rc, n2 = _ws(lib, 1, 16384, 64, 128, 4, 512, opts)
+    assert rc == 0 and 64 << 20 >= n2 - 256 > 0  # bounded by the scratch budget
+    big = _lib.SiOptions(1024, 64, 0, 0, 0)
+    rc, n3 = _ws(lib, 1, 262144, 64, 128, 4, 2048, big)
+    assert rc == 0 and n3 - 256 <= 64 << 20      # independent of S
+    assert _ws(lib, 1, 16383, 64, 128, 4, 512)[0] == -2   # S % m
+    assert _ws(lib, 1, 16384, 48, 128, 4, 512)[0] == -2   # H_I
+    assert _ws(lib, 1, 16384, 64, 96, 4, 512)[0] == -2    # d_I
+    assert _ws(lib, 1, 16384, 64, 128, 4, 0)[0] == -3     # topk
+    assert _ws(lib, 1, 16384, 64, 128, 4, 2049)[0] == -3
+    assert _ws(lib, 1, 16384, 64, 128, 4, 512, _lib.SiOptions(100, 0, 0, 0, 0))[0] == -8
+
+
+def test_null_and_alignment_rejected_before_cuda(lib):
+    P = ctypes.c_void_p
+    ok = P(0x1000)
+    assert lib.si_indexer_topk(None, ok, ok, 1, 64, 8, 64, 4, 8, ok, ok, None) == -1
+    assert lib.si_indexer_topk(P(0x1001), ok, ok, 1, 64, 8, 64, 4, 8, ok, ok, None) == -4
+    assert lib.si_indexer_topk(ok, ok, ok, 1, 64, 8, 64, 4, 9999, ok, ok, None) == -3
+    assert lib.si_topk_scores(None, 1, 4, 4, 1, 2, ok, ok, None, None) == -1
+    assert lib.si_quantize_fp8_rows(ok, 4, 12, ok, ok, None) == -2

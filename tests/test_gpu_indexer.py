@@ -1,0 +1,86 @@
+"""End-to-end indexer step through the C ABI against the fp64 oracle: mean
+recall >= 0.999, exact sets where a row sees <= k keys, every extra key within
+1e-3 * max|row score| of the oracle's k-th score, and the structural
+invariants (order, visibility, count, padding)."""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import streaming_top_lightning_b200 as stl
+from tests import _gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_all_rows():
+    sh = synth.shape("tiny")
+    q, w, kc = _gpu.inputs(sh)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    rows = np.arange(sh.B * sh.S)
+    res = _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    assert res["mean_recall"] == 1.0
+    _gpu.structural(sh, gi, gs, rows)
+
+
+SMALL = [
+    # B, S, m, H, D, k
+    (2, 100, 4, 8, 64, 16),     # S not a multiple of the 32-query tile, 2 batches
+    (1, 256, 2, 16, 128, 32),
+    (1, 520, 4, 32, 64, 40),
+    (2, 1024, 4, 64, 128, 100),
+    (1, 64, 8, 64, 128, 3),     # m=8: the first query tile sees no key at all
+    (1, 1024, 1, 64, 128, 2048),  # k above every row's visible count
+    (1, 3000, 4, 64, 64, 333),  # ragged T (750)
+    (3, 200, 4, 16, 64, 7),
+]
+
+
+@pytest.mark.parametrize("B,S,m,H,D,k", SMALL)
+def test_small_shapes(B, S, m, H, D, k):
+    sh = synth.small(B, S, m, H, D, k, seed=S + H, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=S + H)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    rows = np.arange(B * S)
+    _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    _gpu.structural(sh, gi, gs, rows)
+
+
+@pytest.mark.parametrize("chunk", [128, 256, 1024])
+def test_chunked_equals_unchunked(chunk):
+    """Chunking changes only where the selection happens, not the fp32 scores,
+    so the chunked partition-merge path returns exactly the same result."""
+    sh = synth.small(1, 8192, 4, 64, 128, 256, seed=3, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=3)
+    gi0, gs0 = _gpu.run_bf16(sh, q, w, kc)
+    gi1, gs1 = _gpu.run_bf16(sh, q, w, kc, opts=stl.options(key_chunk=chunk))
+    assert torch.equal(gi0, gi1)
+    assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
+
+
+def test_repeatable():
+    sh = synth.small(1, 4096, 4, 64, 128, 512, seed=4, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=4)
+    a = _gpu.run_bf16(sh, q, w, kc)
+    b = _gpu.run_bf16(sh, q, w, kc)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1].view(torch.int32), b[1].view(torch.int32))
+
+
+def test_v4flash_sampled_rows():
+    sh = synth.shape("v4flash_s16k")
+    q, w, kc = _gpu.inputs(sh)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    g = np.random.default_rng(1)
+    rows = np.union1d(g.choice(sh.S, 384, replace=False), [0, 3, 4, 511, 2047, 2048, sh.S - 1])
+    _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    _gpu.structural(sh, gi, gs, np.arange(0, sh.S, 7))
+
+
+def test_large_s64k_sampled_rows():
+    sh = synth.shape("large_s64k")
+    q, w, kc = _gpu.inputs(sh)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    rows = synth.sample_rows(sh)
+    _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    _gpu.structural(sh, gi, gs, np.arange(0, sh.S, 61))

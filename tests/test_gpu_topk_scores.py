@@ -1,0 +1,76 @@
+"""Selection stage on given fp32 scores: bit-exact (indices and score bits)
+against the oracle, including ties, +-0, +-inf, constant rows, rows with fewer
+visible keys than k, ragged sizes and the chunked partition-merge path."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import streaming_top_lightning_b200 as stl
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # B, S, T, m, k, key_chunk
+    (1, 64, 16, 4, 8, 0),
+    (2, 37, 13, 3, 5, 0),          # ragged: S not a multiple of the query tile
+    (1, 1000, 700, 1, 64, 0),      # T not a multiple of 128
+    (1, 2048, 512, 4, 64, 128),    # chunked: 4 chunks + merge
+    (1, 4096, 1024, 4, 512, 256),
+    (1, 2048, 2048, 1, 2048, 0),   # k at its maximum, many candidates per strip
+    (1, 300, 5000, 1, 2048, 1024), # chunked with k at its maximum
+    (3, 100, 300, 2, 300, 128),    # k > T
+    (1, 5, 3, 1, 1, 0),            # k = 1, tiny
+]
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "const", "inf"])
+@pytest.mark.parametrize("B,S,T,m,k,chunk", CASES)
+def test_bit_exact(kind, B, S, T, m, k, chunk):
+    X = synth.gen_scores(B, S, T, seed=B * 7 + S, kind=kind)
+    opts = stl.options(key_chunk=chunk) if chunk else None
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), m, k, opts=opts)
+    torch.cuda.synchronize()
+    assert stl.device_error() == 0
+    oi, os_ = oracle.topk_scores(X, m, k)
+    gi = gi.reshape(-1, k).cpu().numpy()
+    gs = gs.reshape(-1, k).cpu().numpy()
+    np.testing.assert_array_equal(gi, oi)
+    np.testing.assert_array_equal(gs.view(np.uint32), os_.view(np.uint32))
+
+
+def test_increasing_rows_worst_case():
+    """Scores rising along j: every key beats the running k-th, so every strip
+    overflows the candidate buffer."""
+    B, S, T, m, k = 1, 64, 4096, 1, 1024
+    X = np.broadcast_to(np.arange(T, dtype=np.float32), (B, S, T)).copy()
+    X += np.random.default_rng(0).standard_normal((B, S, T)).astype(np.float32) * 1e-3
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), m, k)
+    oi, os_ = oracle.topk_scores(X, m, k)
+    np.testing.assert_array_equal(gi.reshape(-1, k).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, k).cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
+def test_chunk_sizes_agree():
+    X = synth.gen_scores(1, 512, 3000, seed=5, kind="ties")
+    ref = None
+    for chunk in [0, 128, 384, 1024, 2048]:
+        opts = stl.options(key_chunk=chunk) if chunk else None
+        gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), 1, 700, opts=opts)
+        cur = (gi.cpu().numpy(), gs.cpu().numpy().view(np.uint32))
+        if ref is None:
+            ref = cur
+        np.testing.assert_array_equal(cur[0], ref[0])
+        np.testing.assert_array_equal(cur[1], ref[1])
+
+
+def test_small_scratch_budget_many_blocks():
+    """A 1 MiB scratch budget forces many query blocks; the result is unchanged."""
+    X = synth.gen_scores(2, 256, 2048, seed=9, kind="normal")
+    opts = stl.options(key_chunk=256, scratch_mb=1)
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), 2, 256, opts=opts)
+    oi, os_ = oracle.topk_scores(X, 2, 256)
+    np.testing.assert_array_equal(gi.reshape(-1, 256).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, 256).cpu().numpy().view(np.uint32), os_.view(np.uint32))

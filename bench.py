@@ -259,13 +259,11 @@ def run_native(args, sh):
     idx = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32, device=dev)
     score = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32, device=dev)
     if args.fp8:
-        q8, s_q = stl.quantize_fp8_rows(q_d)
-        k8, s_k = stl.quantize_fp8_rows(kc_d)
-        del q_d
-        q_d = None
-
         def step():
-            stl.indexer_topk_fp8(q8, s_q, w_d, k8, s_k, sh.m, sh.topk, out=(idx, score),
+            # the FP8 step starts from the bf16 inputs: quantise, then score + select
+            a8, s_q = stl.quantize_fp8_rows(q_d)
+            b8, s_k = stl.quantize_fp8_rows(kc_d)
+            stl.indexer_topk_fp8(a8, s_q, w_d, b8, s_k, sh.m, sh.topk, out=(idx, score),
                                  opts=opts, workspace=ws)
     else:
         def step():
@@ -313,6 +311,9 @@ def run_native(args, sh):
 
     # end to end through the public API: host -> device inputs, the call,
     # device -> host result, every step
+    if args.no_e2e:
+        return finish(args, sh, world, rank, P, K, total_ms, launch_ms, None, None, None, None,
+                      peak_alloc, free0, free1, clk, dist)
     idx_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32).pin_memory()
     score_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32).pin_memory()
     qe = torch.empty_like(q_h, device=dev)
@@ -350,7 +351,13 @@ def run_native(args, sh):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     assert stl.device_error() == 0
+    return finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h,
+                  peak_alloc, free0, free1, clk, dist)
 
+
+def finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, peak_alloc,
+           free0, free1, clk, dist):
+    flops_per_pair = 2 * sh.H * sh.D
     ms_per_step = total_ms / K
     value = world * P * sh.B / (ms_per_step / 1e3)
     peaks, peak_src = measured_peaks()
@@ -359,9 +366,11 @@ def run_native(args, sh):
     peak_tf = float(peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
     tflops_step = flops_launch / (ms_per_step / 1e3) / 1e12
     traffic = traffic_record(sh.name, args.fp8)
+    # our kernels per step: the score kernel per query block (+ the merge kernel
+    # when keys are chunked), plus the two quantiser launches on the FP8 path
     launches_per_step = 1 + (1 if args.key_chunk and args.key_chunk < sh.T else 0)
     if args.fp8:
-        launches_per_step += 0
+        launches_per_step += 2
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -379,8 +388,9 @@ def run_native(args, sh):
                      + (" x2 nominal fp8/bf16 ratio" if args.fp8 else ""),
                      "algorithmic_flops_per_launch": flops_launch,
                      "avg_launch_ms": launch_ms},
-        "e2e": {"value": world * P * sh.B * Ke / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": None if e2e_ms is None else {
+            "value": world * P * sh.B * Ke / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": K * launches_per_step,
         "clocks": clk.summary(),
     }
@@ -409,6 +419,7 @@ def main():
     ap.add_argument("--fp8", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     sh = synth.shape(args.workload)
     if args.topk:

@@ -12,6 +12,7 @@
 // keys, units write the final answer directly and no merge pass runs.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "streamindex.h"
@@ -203,7 +204,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
     UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base};
     ScoreParams p{};
-    p.sel = SelParams{B, S, T, m, K, pl.QT, sp_plan.CS, g_lo, n_tiles, pl.nch_max,
+    p.sel = SelParams{B, S, T, m, K, pl.QT, sp_plan.CS, sp_plan.cap, g_lo, n_tiles, pl.nch_max,
                       out_idx, out_score, partial};
     p.ug = ug;
     p.w = w;
@@ -224,6 +225,9 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     if (pl.nch_max > 1 && launch_merge(partial, p.sel, ug, stream) != cudaSuccess)
       return SI_ERR_CUDA;
   }
+  // the selection leaves each row's K best unsorted; order them
+  if (launch_sort_rows(out_idx, out_score, (int64_t)B * S, K, dev->sms, stream) != cudaSuccess)
+    return SI_ERR_CUDA;
   return SI_OK;
 }
 
@@ -353,6 +357,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   if ((rc = dev_info(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int QT = 4, CS = 1024;
+  const int cap = ((std::max(topk + 32, 2 * topk) + 31) / 32) * 32;
   // the selection-only path sees T keys per row; m still sets visibility
   Plan pl{};
   {
@@ -391,7 +396,8 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
     UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base};
-    SelParams sp{B, S, T, m, topk, QT, CS, g_lo, n_tiles, pl.nch_max, out_idx, out_score, partial};
+    SelParams sp{B, S, T, m, topk, QT, CS, cap, g_lo, n_tiles, pl.nch_max, out_idx, out_score,
+                 partial};
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -403,6 +409,9 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
       rc = SI_ERR_CUDA;
     id_base += units + grid;
   }
+  if (rc == SI_OK &&
+      launch_sort_rows(out_idx, out_score, (int64_t)B * S, topk, dev->sms, st) != cudaSuccess)
+    rc = SI_ERR_CUDA;
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;
   return rc;
 }

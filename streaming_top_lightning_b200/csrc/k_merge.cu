@@ -3,117 +3,99 @@
 // "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
 // Top-k", Abstract: a chunked partition-merge top-k driver keeps the indexer
 // from ever holding the full score tensor.  When a query's visible keys span
-// several key chunks, each chunk's unit leaves a sorted partial list of K keys
-// in scratch; this kernel folds them into the final answer.  Under the strict
-// total order of the 64-bit keys, the top K of a union equals the top K of the
-// per-part top Ks, so the result is exactly the top K over all chunks.
+// several key chunks, each chunk's unit leaves a sorted, 0-padded partial list
+// of its K best keys in scratch; this kernel folds them into the final answer.  Under
+// the strict total order of the 64-bit keys, the top K of a union equals the
+// top K of the per-part top Ks, so the result is exactly the top K over all
+// chunks.
 //
-// One CTA per query.  The running list and the next partial list sit in shared
-// memory; each fold is a merge path over 256 threads (8 outputs each) that
-// rebuilds only the positions at or after the first one the partial list
-// takes, staged through registers so it can run in place.
-#include "si_select.cuh"
+// One warp per query, with the same candidate pool, threshold and radix
+// select as the score kernel's selection (si_select.cuh); the result is
+// written unsorted, like the score kernel's, for the row sort that follows.
+#include <algorithm>
+
 #include "si_kernels.h"
 
 namespace si {
 
-constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = 4;
 
-__global__ void __launch_bounds__(kMergeThreads)
-    k_merge(const uint64_t* __restrict__ partial, SelParams sp, UnitGrid ug) {
+// Append the keys of one partial list that beat theta.
+SI_DEV void pool_take_keys(const uint64_t* keys, int n, uint64_t* pool, int cap, int K, int& np,
+                           uint64_t& theta, uint32_t* hist, int lane) {
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int r0 = 0; r0 < n; r0 += 32) {
+    const int r = r0 + lane;
+    const uint64_t key = r < n ? keys[r] : 0ull;
+    bool take = key > theta;
+    uint32_t mask = __ballot_sync(0xFFFFFFFFu, take);
+    if (mask == 0u) continue;
+    int cnt = __popc(mask);
+    if (np + cnt > cap) {
+      __syncwarp();
+      uint64_t th = theta;
+      if (!pool_prune(pool, &np, K, &th, lane) || np + 32 > cap) {
+        th = pool_shrink(pool, np, K, hist, lane);
+        np = K;
+      }
+      theta = th;
+      take = take && key > theta;
+      mask = __ballot_sync(0xFFFFFFFFu, take);
+      cnt = __popc(mask);
+    }
+    if (take) pool[np + __popc(mask & lt_mask)] = key;
+    np += cnt;
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    k_merge(const uint64_t* __restrict__ partial, SelParams sp, UnitGrid ug, int cap) {
   extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = sp.K, QT = sp.QT;
-  int cta = blockIdx.x;
-  const int qi = cta % QT;
-  cta /= QT;
-  const int gl = cta % sp.n_tiles;
-  const int b = cta / sp.n_tiles;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem) + warp * 256;
+  uint64_t* pool = reinterpret_cast<uint64_t*>(smem + sizeof(uint32_t) * kMergeWarps * 256) +
+                   (size_t)warp * cap;
+  const int64_t qid = (int64_t)blockIdx.x * kMergeWarps + warp;
+  if (qid >= (int64_t)sp.B * sp.n_tiles * QT) return;
+  const int qi = (int)(qid % QT);
+  const int gl = (int)((qid / QT) % sp.n_tiles);
+  const int b = (int)(qid / ((int64_t)QT * sp.n_tiles));
   const int g = sp.g_lo + gl;
   const int t = g * QT + qi;
   if (t >= sp.S) return;
   const int nch = tile_chunks(ug, g);
   if (nch <= 1) return;
 
-  uint64_t* L = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* C = L + K;
-  __shared__ int s_f;
-  const int tid = threadIdx.x;
   const uint64_t* base = partial + (((int64_t)b * sp.n_tiles + gl) * sp.nch_max) * QT * K;
-  auto list = [&](int c) { return base + ((int64_t)c * QT + qi) * K; };
-
-  for (int r = tid; r < K; r += kMergeThreads) L[r] = list(0)[r];
-  for (int c = 1; c < nch; ++c) {
-    const uint64_t* src = list(c);
-    for (int r = tid; r < K; r += kMergeThreads) C[r] = src[r];
-    __syncthreads();
-    if (tid == 0) {
-      const uint64_t c0 = C[0];
-      int lo = 0, hi = K;
-      if (c0 == 0ull) {
-        lo = K;  // empty partial list: nothing to fold
-      } else {
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (L[mid] > c0) lo = mid + 1;
-          else hi = mid;
-        }
-      }
-      s_f = lo;
-    }
-    __syncthreads();
-    const int f = s_f;
-    uint64_t* A = L + f;
-    const int na = K - f;
-    const int n = K;
-    constexpr int R = kMergeR, P = kMergeThreads * R;
-    for (int ph = (na + P - 1) / P - 1; ph >= 0; --ph) {
-      const int d = ph * P + tid * R;
-      uint64_t v[R];
-      if (d < na) {
-        int l2 = d - n > 0 ? d - n : 0;
-        int h2 = d < na ? d : na;
-        while (l2 < h2) {
-          const int mid = (l2 + h2) >> 1;
-          if (A[mid] > C[d - 1 - mid]) l2 = mid + 1;
-          else h2 = mid;
-        }
-        int ia = l2, ib = d - l2;
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          if (d + r < na) {
-            const bool take_a = (ib >= n) || (ia < na && A[ia] > C[ib]);
-            v[r] = take_a ? A[ia] : C[ib];
-            ia += take_a ? 1 : 0;
-            ib += take_a ? 0 : 1;
-          }
-        }
-      }
-      __syncthreads();
-      if (d < na) {
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-          if (d + r < na) A[d + r] = v[r];
-      }
-      __syncthreads();
-    }
-  }
-  __syncthreads();
+  int np = 0;
+  uint64_t theta = 0ull;
+  for (int c = 0; c < nch; ++c)
+    pool_take_keys(base + ((int64_t)c * QT + qi) * K, K, pool, cap, K, np, theta, hist, lane);
+  const int n = pool_finish(pool, np, K, hist, lane);
   const int64_t o = ((int64_t)b * sp.S + t) * K;
-  for (int r = tid; r < K; r += kMergeThreads) {
-    const uint64_t k = L[r];
-    sp.out_idx[o + r] = k ? key_index(k) : -1;
-    sp.out_score[o + r] = k ? key_score(k) : __int_as_float(0xFF800000);
+  for (int r = lane; r < K; r += 32) {
+    const bool real = r < n;
+    const uint64_t k = real ? pool[r] : 0ull;
+    sp.out_idx[o + r] = real ? key_index(k) : -1;
+    sp.out_score[o + r] = real ? key_score(k) : __int_as_float(0xFF800000);
   }
 }
 
 cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                          cudaStream_t stream) {
-  const size_t smem = sizeof(uint64_t) * 2 * sp.K;
+  // pool room: twice K keeps radix selects rare, and at least one block of
+  // 32 beyond K
+  const int K = sp.K;
+  const int cap = ((std::max(K + 32, 2 * K) + 31) / 32) * 32;
+  const size_t smem = sizeof(uint32_t) * kMergeWarps * 256 + sizeof(uint64_t) * kMergeWarps * cap;
   cudaError_t e =
       cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int grid = ug.B * sp.n_tiles * sp.QT;
-  k_merge<<<grid, kMergeThreads, smem, stream>>>(partial, sp, ug);
+  const int64_t queries = (int64_t)ug.B * sp.n_tiles * sp.QT;
+  const int grid = (int)((queries + kMergeWarps - 1) / kMergeWarps);
+  k_merge<<<grid, kMergeWarps * 32, smem, stream>>>(partial, sp, ug, cap);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,8 @@
 //   warps 6-9  streaming selection (si_select.cuh) on the strips.
 // Every wait is bounded (si_common.cuh); on expiry the CTA drains its own
 // asynchronous copies and MMAs, frees TMEM and exits with an error word set.
+#include <algorithm>
+
 #include "si_kernels.h"
 
 namespace si {
@@ -107,15 +109,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const SelParams& sp = p.sel;
-  const int K = sp.K, CS = sp.CS, NST = p.nst;
+  const int CS = sp.CS, NST = p.nst;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   uint8_t* q_s = smem;
   uint8_t* kc_s = q_s + G::kQBytes;
   float* strip = reinterpret_cast<float*>(kc_s + (size_t)NST * G::kKcBytes);
-  uint64_t* lists = reinterpret_cast<uint64_t*>(strip + 2 * QT * CS);
-  uint64_t* cand = lists + (size_t)QT * K;
-  float* w_s = reinterpret_cast<float*>(cand + kSelWarps * kCandCap);  // [4 warps][kN]
+  uint8_t* sel_base = reinterpret_cast<uint8_t*>(strip + 2 * QT * CS);
+  SelSmem sm;
+  sel_state_carve(sel_base, QT, sp.cap, sm);
+  float* w_s = reinterpret_cast<float*>(sel_base + sel_state_bytes(QT, sp.cap));  // [4][kN]
   ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + 4 * kN);
 
   const uint32_t q_addr = smem_u32(q_s), kc_addr = smem_u32(kc_s);
@@ -140,7 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     cs->abort = 0u;
     mbar_fence_init();
   }
-  for (int i = tid; i < QT * K; i += kThreads) lists[i] = 0ull;
+  if (tid < QT) {
+    sm.npool[tid] = 0;
+    sm.theta[tid] = 0ull;
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(&cs->tmem_base), 512);
     tmem_relinquish();
@@ -395,8 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- selection
-    SelSmem sm{lists, cand, strip, cs->meta, smem_u32(&cs->strip_full[0]),
-               smem_u32(&cs->strip_empty[0])};
+    sm.strip = strip;
+    sm.meta = cs->meta;
+    sm.full_bar = smem_u32(&cs->strip_full[0]);
+    sm.empty_bar = smem_u32(&cs->strip_empty[0]);
     select_loop(sp, sm, ctl, warp - kSelWarp0, lane);
   }
 
@@ -443,32 +451,52 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
   return cudaErrorInvalidValue;
 }
 
+// Shared-memory plan: the query tile, NST key-tile stages, two score strips of
+// CS keys per query, the selection pools (cap keys per query) and the small
+// control block.  Candidates are ranked lexicographically: a pool of at least
+// 1.5K keys first (fewer radix selects), then 3 stages, then strips of 512
+// keys, then the larger pool and more stages.
 ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
-  ScorePlan pl{};
+  ScorePlan best{};
+  best.ok = false;
   const int esz = fp8 ? 1 : 2;
   const int QT = kN / H;
   const size_t q_bytes = (size_t)kN * D * esz;
   const size_t kc_bytes = (size_t)kM * D * esz;
-  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(uint64_t) * QT * K +
-                       sizeof(uint64_t) * kSelWarps * kCandCap + sizeof(float) * 4 * kN +
+  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * 4 * kN +
                        sizeof(ScoreCtlSmem);
-  pl.QT = QT;
-  pl.ok = false;
-  // prefer long strips, but keep at least 3 pipeline stages when possible
-  for (int min_st = 3; min_st >= 2 && !pl.ok; --min_st) {
-    for (int cs = 1024; cs >= kM; cs >>= 1) {
-      const size_t strip = sizeof(float) * 2 * QT * cs;
-      if (fixed + strip + min_st * kc_bytes > (size_t)max_smem) continue;
-      int nst = (int)((max_smem - fixed - strip) / kc_bytes);
-      if (nst > 6) nst = 6;
-      pl.CS = cs;
-      pl.nst = nst;
-      pl.smem = fixed + strip + nst * kc_bytes;
-      pl.ok = true;
-      break;
+  const int cap_min = ((std::max(K + 32, 64) + 31) / 32) * 32;
+  const int cap_max = ((2 * K + 31) / 32) * 32 > cap_min ? ((2 * K + 31) / 32) * 32 : cap_min;
+  const int cs_max = std::min(1024, std::max(128, 4096 / QT));
+  long best_score[5] = {-1, -1, -1, -1, -1};
+  for (int nst = 2; nst <= 6; ++nst) {
+    for (int cs = 128; cs <= cs_max; cs <<= 1) {
+      const size_t used = fixed + nst * kc_bytes + sizeof(float) * 2 * QT * cs;
+      if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
+      int cap = cap_min;
+      while (cap + 32 <= cap_max && used + sel_state_bytes(QT, cap + 32) <= (size_t)max_smem)
+        cap += 32;
+      const long sc[5] = {std::min(cap, (3 * K) / 2), std::min(nst, 3), std::min(cs, 512), cap,
+                          nst};
+      bool better = false;
+      for (int i = 0; i < 5; ++i) {
+        if (sc[i] != best_score[i]) {
+          better = sc[i] > best_score[i];
+          break;
+        }
+      }
+      if (better) {
+        for (int i = 0; i < 5; ++i) best_score[i] = sc[i];
+        best.QT = QT;
+        best.CS = cs;
+        best.nst = nst;
+        best.cap = cap;
+        best.smem = used + sel_state_bytes(QT, cap);
+        best.ok = true;
+      }
     }
   }
-  return pl;
+  return best;
 }
 
 }  // namespace si

@@ -27,14 +27,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int QT = sp.QT, K = sp.K, CS = sp.CS;
+  const int QT = sp.QT, CS = sp.CS;
 
-  // carve shared memory
+  // carve shared memory: selection state, strips, metadata, barriers
+  SelSmem sm;
   uint8_t* p = smem;
-  uint64_t* lists = reinterpret_cast<uint64_t*>(p);
-  p += sizeof(uint64_t) * QT * K;
-  uint64_t* cand = reinterpret_cast<uint64_t*>(p);
-  p += sizeof(uint64_t) * kSelWarps * kCandCap;
+  sel_state_carve(p, QT, sp.cap, sm);
+  p += sel_state_bytes(QT, sp.cap);
   float* strip = reinterpret_cast<float*>(p);
   p += sizeof(float) * 2 * QT * CS;
   StripMeta* meta = reinterpret_cast<StripMeta*>(p);
@@ -52,11 +51,17 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     misc->abort = 0u;
     mbar_fence_init();
   }
-  for (int i = tid; i < QT * K; i += kTopkThreads) lists[i] = 0ull;
+  for (int i = tid; i < QT; i += kTopkThreads) {
+    sm.npool[i] = 0;
+    sm.theta[i] = 0ull;
+  }
   __syncthreads();
 
   Ctl ctl{err, &misc->abort, timeout_ns};
-  SelSmem sm{lists, cand, strip, meta, full_bar, empty_bar};
+  sm.strip = strip;
+  sm.meta = meta;
+  sm.full_bar = full_bar;
+  sm.empty_bar = empty_bar;
 
   if (warp >= kLoadThreads / 32) {
     select_loop(sp, sm, ctl, warp - kLoadThreads / 32, lane);
@@ -113,16 +118,15 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   __syncthreads();
 }
 
-size_t topk_scores_smem_bytes(int QT, int K, int CS) {
-  return sizeof(uint64_t) * QT * K + sizeof(uint64_t) * kSelWarps * kCandCap +
-         sizeof(float) * 2 * QT * CS + sizeof(StripMeta) * 2 + sizeof(uint64_t) * 4 +
-         sizeof(TopkScoresSmem) + 64;
+size_t topk_scores_smem_bytes(int QT, int cap, int CS) {
+  return sel_state_bytes(QT, cap) + sizeof(float) * 2 * QT * CS + sizeof(StripMeta) * 2 +
+         sizeof(uint64_t) * 4 + sizeof(TopkScoresSmem) + 64;
 }
 
 cudaError_t launch_topk_scores(const float* X, const SelParams& sp, const UnitGrid& ug,
                                int* counter, uint32_t* err, uint64_t timeout_ns, int grid,
                                cudaStream_t stream) {
-  const size_t smem = topk_scores_smem_bytes(sp.QT, sp.K, sp.CS);
+  const size_t smem = topk_scores_smem_bytes(sp.QT, sp.cap, sp.CS);
   cudaError_t e = cudaFuncSetAttribute(k_topk_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

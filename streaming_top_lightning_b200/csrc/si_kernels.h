@@ -28,6 +28,7 @@ struct ScorePlan {
   int QT;        // queries per tile (256 / H)
   int CS;        // keys per score strip
   int nst;       // pipeline stages
+  int cap;       // selection pool entries per query
   size_t smem;   // dynamic shared memory bytes
   bool ok;
 };
@@ -38,13 +39,18 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
                               size_t smem, cudaStream_t stream);
 
-size_t topk_scores_smem_bytes(int QT, int K, int CS);
+size_t topk_scores_smem_bytes(int QT, int cap, int CS);
 cudaError_t launch_topk_scores(const float* X, const SelParams& sp, const UnitGrid& ug,
                                int* counter, uint32_t* err, uint64_t timeout_ns, int grid,
                                cudaStream_t stream);
 
 cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                          cudaStream_t stream);
+
+// Sorts each of the rows [rows, K] of (idx, score) in place into the output
+// order (score descending, index ascending, padding last).
+cudaError_t launch_sort_rows(int32_t* idx, float* score, int64_t rows, int K, int sms,
+                             cudaStream_t stream);
 
 cudaError_t launch_quantize_fp8(const uint16_t* x, int64_t rows, int cols, uint8_t* x8,
                                 float* scale, cudaStream_t stream);

@@ -5,22 +5,24 @@
 // "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
 // Top-k", Abstract: the top-k keys are selected per query by a chunked
 // partition-merge driver that never holds the full score tensor.  Here each
-// query owns a running list of its best K keys so far (sorted, 64-bit keys
-// from si_common.cuh, 0 = empty) in shared memory.  Scores are consumed in
-// strips of up to CS keys: a key enters a warp-private candidate buffer only if
-// it beats the list's current K-th entry; full buffers are bitonic-sorted by
-// the warp and merged into the list in place (merge path, back to front).  A
-// unit (a tile of QT queries x one key chunk) ends by writing each list out,
-// either as the final answer or as a partial list for the merge kernel.
+// query owns an unsorted candidate pool (64-bit keys from si_common.cuh) in
+// shared memory and a threshold theta, the K-th best key seen so far (0 until
+// K keys have been seen).  Scores arrive in strips of up to CS keys; a key
+// enters the pool only if it beats theta.  When the pool is full, a warp radix
+// select finds the exact K-th largest pool key, which becomes theta, and the
+// pool is compacted to the K keys at or above it.  A unit (a tile of QT
+// queries x one key chunk) ends with one last select; the K survivors are
+// written out unsorted, either as the final answer or as a partial list for
+// the merge kernel, and a separate pass (k_sort_rows.cu) orders the rows.
+// Every pass reads the pool with consecutive lanes on consecutive keys, so no
+// access has bank conflicts.
 #pragma once
 
 #include "si_common.cuh"
 
 namespace si {
 
-constexpr int kSelWarps = 4;    // selection warps per CTA
-constexpr int kCandCap = 256;   // candidate buffer entries per selection warp
-constexpr int kMergeR = 8;      // outputs per lane per merge phase
+constexpr int kSelWarps = 4;  // selection warps per CTA
 
 // What a filled strip slot carries from its producer to the selection warps.
 struct StripMeta {
@@ -34,16 +36,19 @@ struct StripMeta {
 
 struct SelParams {
   int B, S, T, m, K, QT, CS;
+  int cap;             // pool entries per query (>= K + 32)
   int g_lo, n_tiles;   // query tiles [g_lo, g_lo + n_tiles) in this launch
   int nch_max;         // chunk slots per query tile in the partial scratch
   int32_t* out_idx;    // [B,S,K]
   float* out_score;    // [B,S,K]
-  uint64_t* partial;   // [B, n_tiles, nch_max, QT, K] sorted keys
+  uint64_t* partial;   // [B, n_tiles, nch_max, QT, K] selected keys, 0-padded
 };
 
 struct SelSmem {
-  uint64_t* lists;     // [QT][K]
-  uint64_t* cand;      // [kSelWarps][kCandCap]
+  uint64_t* pool;      // [QT][cap] candidate keys
+  uint64_t* theta;     // [QT] current threshold
+  int* npool;          // [QT] keys in each pool
+  uint32_t* hist;      // [kSelWarps][8][32] digit counters of each selection warp
   float* strip;        // [2][QT][CS]
   StripMeta* meta;     // [2]
   uint32_t full_bar;   // 2 mbarriers, 8 bytes apart
@@ -55,149 +60,281 @@ SI_DEV int visible_keys(int t, int T, int m) {
   return v < T ? v : T;
 }
 
-// Bitonic sort of a[0, n2) into descending order by one warp (n2 a power of 2).
-SI_DEV void warp_sort_desc(uint64_t* a, int n2, int lane) {
-  for (int size = 2; size <= n2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = lane; i < (n2 >> 1); i += 32) {
-        const int lo = ((i & ~(stride - 1)) << 1) | (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const uint64_t x = a[lo], y = a[hi];
-        if ((x < y) == up) {
-          a[lo] = y;
-          a[hi] = x;
-        }
+__host__ __device__ constexpr int pow2ceil(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// ------------------------------------------------------------------ radix select
+// Compacts pool[0, np) (np > K, distinct keys) in place to its K largest keys
+// and returns the smallest of them.  MSD radix select on 5-bit digits,
+// starting at the highest bit where the pool keys differ.  Each lane counts
+// the digits of its own keys (every 32nd key) in eight registers of four byte
+// counters (digit d in byte d%4 of register d/4), with predicated adds and no
+// memory traffic; the counters then go to shared memory as hist[d/4][lane],
+// one transposed pass sums lane v's digit v over all lanes, and a suffix sum
+// across lanes names the digit bucket that holds the K-th largest key.  It
+// stops once a whole bucket is taken; one last pass keeps every key whose
+// high bits reach the prefix.  hist: this warp's 8 x 32 words.
+// Requires np <= 255 * 32 (byte counters).
+static __device__ __noinline__ uint64_t pool_shrink(uint64_t* pool, int np, int K, uint32_t* hist,
+                                             int lane) {
+  uint64_t all_and = ~0ull, any_or = 0ull;
+  {
+    int i = lane;
+    for (; i + 96 < np; i += 128) {
+      const uint64_t k0 = pool[i], k1 = pool[i + 32], k2 = pool[i + 64], k3 = pool[i + 96];
+      all_and &= k0 & k1 & k2 & k3;
+      any_or |= k0 | k1 | k2 | k3;
+    }
+    for (; i < np; i += 32) {
+      const uint64_t k = pool[i];
+      all_and &= k;
+      any_or |= k;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    all_and &= __shfl_xor_sync(0xFFFFFFFFu, all_and, o);
+    any_or |= __shfl_xor_sync(0xFFFFFFFFu, any_or, o);
+  }
+  const uint64_t diff = all_and ^ any_or;  // nonzero: keys are distinct, np >= 2
+  int top = 63 - __clzll((long long)diff);
+  // bits above `top` are common to every key; there are none when top is 63
+  uint64_t prefix = (top >= 63) ? 0ull : (all_and & ~((2ull << top) - 1ull));
+  uint32_t need = (uint32_t)K;
+  int lo_bit = 0;
+  for (;;) {
+    const int width = top + 1 < 5 ? top + 1 : 5;
+    lo_bit = top - width + 1;
+    const uint64_t hi_mask = (top >= 63) ? 0ull : ~((2ull << top) - 1ull);
+    const uint32_t dmask = (1u << width) - 1u;
+    uint32_t c[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    for (int i = lane; i < np; i += 32) {
+      const uint64_t k = pool[i];
+      const uint32_t d = (uint32_t)(k >> lo_bit) & dmask;
+      const uint32_t inc = ((k & hi_mask) == prefix) ? (1u << ((d & 3u) * 8u)) : 0u;
+      const uint32_t row = d >> 2;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) c[r] += (row == (uint32_t)r) ? inc : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) hist[r * 32 + lane] = c[r];
+    __syncwarp();
+    uint32_t cnt = 0;
+    if ((uint32_t)lane <= dmask) {
+      const uint32_t* row = hist + (lane >> 2) * 32;
+      const uint32_t sh = (lane & 3) * 8;
+#pragma unroll 8
+      for (int l = 0; l < 32; ++l) cnt += (row[(l + lane) & 31] >> sh) & 255u;
+    }
+    __syncwarp();
+    uint32_t suf = cnt;  // keys with digit >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+      if (lane + o < 32) suf += y;
+    }
+    const uint32_t above = suf - cnt;
+    const uint32_t here = __ballot_sync(0xFFFFFFFFu, cnt > 0u && above < need && need <= suf);
+    const int dstar = __ffs(here) - 1;
+    const uint32_t a = __shfl_sync(0xFFFFFFFFu, above, dstar);
+    const uint32_t cb = __shfl_sync(0xFFFFFFFFu, cnt, dstar);
+    prefix |= (uint64_t)dstar << lo_bit;
+    need -= a;
+    if (cb == need || lo_bit == 0) break;
+    top = lo_bit - 1;
+  }
+  const uint64_t pre_hi = prefix >> lo_bit;
+  uint64_t mn = ~0ull;
+  int w = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  // in place, forward: a block's keys are all read before any is written, and
+  // the write position w + rank never passes the read position
+  for (int i0 = 0; i0 < np; i0 += 64) {
+    const int i = i0 + lane;
+    const uint64_t ka = i < np ? pool[i] : 0ull;
+    const uint64_t kb = i + 32 < np ? pool[i + 32] : 0ull;
+    const bool ta = i < np && (ka >> lo_bit) >= pre_hi;
+    const bool tb = i + 32 < np && (kb >> lo_bit) >= pre_hi;
+    const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta);
+    const uint32_t mb = __ballot_sync(0xFFFFFFFFu, tb);
+    if (ta) {
+      pool[w + __popc(ma & lt_mask)] = ka;
+      mn = ka < mn ? ka : mn;
+    }
+    w += __popc(ma);
+    if (tb) {
+      pool[w + __popc(mb & lt_mask)] = kb;
+      mn = kb < mn ? kb : mn;
+    }
+    w += __popc(mb);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+    mn = y < mn ? y : mn;
+  }
+  __syncwarp();
+  return mn;
+}
+
+// ------------------------------------------------------------------ pruning
+// Cheap mid-stream shrink.  pool[0, np) holds np > K distinct keys.  Each
+// lane samples one key (evenly spread over the pool, which is in arrival
+// order), the warp sorts the 32 samples (bitonic, one key per lane, xor
+// shuffles) and takes as pivot the sample whose rank predicts about
+// target = K + K/8 + 32 pool keys at or above it.  The keys at or above the
+// pivot are counted; if fewer than K, a lower sample is tried.  The pool is
+// then compacted to the c >= K keys at or above the pivot, and the pivot
+// becomes the new threshold: it is a pool key with at least K keys at or
+// above it, so no key below it can be among the K best.  Returns false (pool
+// unchanged) if even the lowest sample leaves fewer than K keys.
+static __device__ __noinline__ bool pool_prune(uint64_t* pool, int* np_io, int K, uint64_t* theta_out,
+                                        int lane) {
+  const int np = *np_io;
+  uint64_t v = pool[(int)(((long long)(2 * lane + 1) * np) >> 6)];
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int s = size >> 1; s > 0; s >>= 1) {
+      const bool dir = (lane & size) == 0;  // lower lane keeps the max
+      const bool lower = (lane & s) == 0;
+      const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, v, s);
+      const bool gt = v > y;
+      v = ((lower == dir) == gt) ? v : y;
+    }
+  }
+  // v is now the sample of rank `lane` (0 = largest)
+  const long long target = (long long)K + K / 8 + 32;
+  int r = (int)((32ll * target + np - 1) / np) - 1;
+  if (r < 0) r = 0;
+  for (; r < 32; r += 2) {
+    const uint64_t pivot = __shfl_sync(0xFFFFFFFFu, v, r);
+    int c = 0;
+    for (int i = lane; i < np; i += 32) c += pool[i] >= pivot ? 1 : 0;
+    c = __reduce_add_sync(0xFFFFFFFFu, c);
+    if (c >= K) {
+      if (c >= np) return false;  // nothing to drop
+      int w = 0;
+      const uint32_t lt_mask = (1u << lane) - 1u;
+      for (int i0 = 0; i0 < np; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t k = i < np ? pool[i] : 0ull;
+        const bool take = i < np && k >= pivot;
+        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, take);
+        if (take) pool[w + __popc(tm & lt_mask)] = k;  // forward, in place
+        w += __popc(tm);
       }
       __syncwarp();
+      *np_io = w;
+      *theta_out = pivot;
+      return true;
     }
   }
+  return false;
 }
 
-// L[0, K) sorted descending; C[0, n) sorted descending, n >= 1, all keys
-// distinct.  Replaces L by the K largest keys of L and C, in place.
-// Positions before the first one C[0] would take are unchanged.  The rest is
-// rebuilt by merge path in phases from the back: a phase reads only list
-// entries at or below its own output range, and no later phase reads that
-// range, so staging each phase's outputs in registers makes it safe in place.
-SI_DEV void warp_merge_into(uint64_t* L, int K, const uint64_t* C, int n, int lane) {
-  const uint64_t c0 = C[0];
-  int lo = 0, hi = K;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (L[mid] > c0) lo = mid + 1;
-    else hi = mid;
-  }
-  const int f = lo;
-  if (f >= K) return;
-  uint64_t* A = L + f;
-  const int na = K - f;  // also the number of outputs rebuilt
-  constexpr int P = 32 * kMergeR;
-  for (int ph = (na + P - 1) / P - 1; ph >= 0; --ph) {
-    const int d = ph * P + lane * kMergeR;
-    uint64_t v[kMergeR];
-    if (d < na) {
-      int l2 = d - n > 0 ? d - n : 0;
-      int h2 = d < na ? d : na;
-      while (l2 < h2) {
-        const int mid = (l2 + h2) >> 1;
-        if (A[mid] > C[d - 1 - mid]) l2 = mid + 1;
-        else h2 = mid;
-      }
-      int ia = l2, ib = d - l2;
-#pragma unroll
-      for (int r = 0; r < kMergeR; ++r) {
-        if (d + r < na) {
-          const bool take_a = (ib >= n) || (ia < na && A[ia] > C[ib]);
-          v[r] = take_a ? A[ia] : C[ib];
-          ia += take_a ? 1 : 0;
-          ib += take_a ? 0 : 1;
-        }
-      }
-    }
-    __syncwarp();
-    if (d < na) {
-#pragma unroll
-      for (int r = 0; r < kMergeR; ++r)
-        if (d + r < na) A[d + r] = v[r];
-    }
-    __syncwarp();
-  }
-}
-
-SI_DEV void warp_flush(uint64_t* L, int K, uint64_t* cb, int n, int lane) {
-  __syncwarp();
-  int n2 = 2;
-  while (n2 < n) n2 <<= 1;
-  for (int i = n + lane; i < n2; i += 32) cb[i] = 0ull;
-  __syncwarp();
-  warp_sort_desc(cb, n2, lane);
-  warp_merge_into(L, K, cb, n, lane);
-  __syncwarp();
-}
-
+// ------------------------------------------------------------------ strips
 // Consume one strip of scores for one query: keys j0 + p, p < nkeys; only
-// keys j < V are visible.
-SI_DEV void warp_take_strip(const float* st, int j0, int nkeys, int V, uint64_t* L, int K,
-                            uint64_t* cb, int lane) {
+// keys j < V are visible.  Keys above theta join the pool; a full pool is
+// shrunk to its K best by pool_shrink, which also raises theta.
+SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t* pool, int cap,
+                            int K, int* np_p, uint64_t* th_p, uint32_t* hist, int lane) {
   int lim = V - j0;
   if (lim > nkeys) lim = nkeys;
   if (lim <= 0) return;
-  uint64_t theta = L[K - 1];
-  int nc = 0;
+  uint64_t theta = *th_p;
+  int np = *np_p;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int p0 = 0; p0 < lim; p0 += 32) {
-    const int p = p0 + lane;
-    uint64_t key = 0ull;
-    bool take = false;
-    if (p < lim) {
-      key = make_key(st[p], j0 + p);
-      take = key > theta;
+  for (int p0 = 0; p0 < lim; p0 += 128) {
+    // four independent groups of 32 keys per round
+    uint64_t key[4];
+    bool take[4];
+    uint32_t mask[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = p0 + 32 * u + lane;
+      key[u] = p < lim ? make_key(st[p], j0 + p) : 0ull;
+      take[u] = p < lim && key[u] > theta;
     }
-    uint32_t mask = __ballot_sync(0xFFFFFFFFu, take);
-    if (mask == 0u) continue;
-    int cnt = __popc(mask);
-    if (nc + cnt > kCandCap) {
-      warp_flush(L, K, cb, nc, lane);
-      nc = 0;
-      theta = L[K - 1];
-      take = take && key > theta;
-      mask = __ballot_sync(0xFFFFFFFFu, take);
-      cnt = __popc(mask);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) mask[u] = __ballot_sync(0xFFFFFFFFu, take[u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (mask[u] == 0u) continue;
+      int cnt = __popc(mask[u]);
+      if (np + cnt > cap) {
+        __syncwarp();
+        uint64_t th = theta;
+        if (!pool_prune(pool, &np, K, &th, lane) || np + 32 > cap) {
+          th = pool_shrink(pool, np, K, hist, lane);
+          np = K;
+        }
+        theta = th;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          take[v] = take[v] && key[v] > theta;
+          mask[v] = __ballot_sync(0xFFFFFFFFu, take[v]);
+        }
+        cnt = __popc(mask[u]);
+      }
+      if (take[u]) pool[np + __popc(mask[u] & lt_mask)] = key[u];
+      np += cnt;
     }
-    if (take) cb[nc + __popc(mask & lt_mask)] = key;
-    nc += cnt;
   }
-  if (nc > 0) warp_flush(L, K, cb, nc, lane);
+  __syncwarp();
+  if (lane == 0) {
+    *np_p = np;
+    *th_p = theta;
+  }
+  __syncwarp();
 }
 
-// Write one query's list out and clear it for the next unit.
-SI_DEV void warp_emit(const SelParams& p, const StripMeta& md, int qi, uint64_t* L, int lane) {
+// Final select of a query's pool: afterwards pool[0, n) holds its n = min(np, K)
+// best keys, in no particular order (the output rows are sorted afterwards by
+// a separate pass over the result).
+SI_DEV int pool_finish(uint64_t* pool, int np, int K, uint32_t* hist, int lane) {
+  __syncwarp();
+  if (np > K) {
+    uint64_t th;
+    while (np > K + K / 4 + 64 && pool_prune(pool, &np, K, &th, lane)) {
+    }
+    pool_shrink(pool, np, K, hist, lane);
+    np = K;
+  }
+  __syncwarp();
+  return np;
+}
+
+// Write one query's selected keys out (final answer or partial list), unsorted.
+SI_DEV void warp_emit(const SelParams& p, const StripMeta& md, int qi, const uint64_t* keys,
+                      int n, int lane) {
   const int t = md.g * p.QT + qi;
   if (md.direct) {
     const int64_t base = ((int64_t)md.b * p.S + t) * p.K;
     for (int r = lane; r < p.K; r += 32) {
-      const uint64_t k = L[r];
-      p.out_idx[base + r] = k ? key_index(k) : -1;
-      p.out_score[base + r] = k ? key_score(k) : __int_as_float(0xFF800000);
-      L[r] = 0ull;
+      const bool real = r < n;
+      const uint64_t k = real ? keys[r] : 0ull;
+      p.out_idx[base + r] = real ? key_index(k) : -1;
+      p.out_score[base + r] = real ? key_score(k) : __int_as_float(0xFF800000);
     }
   } else {
     const int64_t slot =
         (((int64_t)md.b * p.n_tiles + (md.g - p.g_lo)) * p.nch_max + md.c) * p.QT + qi;
     uint64_t* dst = p.partial + slot * p.K;
-    for (int r = lane; r < p.K; r += 32) {
-      dst[r] = L[r];
-      L[r] = 0ull;
-    }
+    for (int r = lane; r < p.K; r += 32) dst[r] = r < n ? keys[r] : 0ull;
   }
   __syncwarp();
 }
 
 // The selection warps' loop: take filled strips in order until a strip says
-// there is no more work (or the CTA aborts).
+// there is no more work (or the CTA aborts).  Query qi belongs to selection
+// warp qi % kSelWarps for the whole kernel, so its pool, threshold and count
+// are only ever touched by that warp.
 SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, int sw, int lane) {
-  uint64_t* cb = sm.cand + sw * kCandCap;
+  uint32_t* hist = sm.hist + sw * 256;
   for (uint32_t it = 0;; ++it) {
     const int slot = it & 1;
     const uint32_t ph = (it >> 1) & 1u;
@@ -208,14 +345,37 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
     for (int qi = sw; qi < p.QT; qi += kSelWarps) {
       const int t = md.g * p.QT + qi;
       if (t >= p.S) continue;
-      uint64_t* L = sm.lists + (size_t)qi * p.K;
-      warp_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), L, p.K,
-                      cb, lane);
-      if (md.last) warp_emit(p, md, qi, L, lane);
+      uint64_t* pool = sm.pool + (size_t)qi * p.cap;
+      pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), pool,
+                      p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane);
+      if (md.last) {
+        const int n = pool_finish(pool, sm.npool[qi], p.K, hist, lane);
+        warp_emit(p, md, qi, pool, n, lane);
+        if (lane == 0) {
+          sm.npool[qi] = 0;
+          sm.theta[qi] = 0ull;
+        }
+        __syncwarp();
+      }
     }
     __syncwarp();
     mbar_arrive(sm.empty_bar + 8 * slot);
   }
+}
+
+// Shared-memory bytes of the selection state for QT queries (pools,
+// thresholds, counts, digit counters), 16-byte aligned.
+__host__ __device__ constexpr size_t sel_state_bytes(int QT, int cap) {
+  return ((sizeof(uint64_t) * (size_t)QT * cap + sizeof(uint64_t) * QT + sizeof(int) * QT +
+           sizeof(uint32_t) * kSelWarps * 256) + 15) & ~(size_t)15;
+}
+
+// Carve the selection state out of shared memory at p (16-byte aligned).
+SI_DEV void sel_state_carve(uint8_t* p, int QT, int cap, SelSmem& sm) {
+  sm.pool = reinterpret_cast<uint64_t*>(p);
+  sm.theta = sm.pool + (size_t)QT * cap;
+  sm.npool = reinterpret_cast<int*>(sm.theta + QT);
+  sm.hist = reinterpret_cast<uint32_t*>(sm.npool + QT);
 }
 
 // ------------------------------------------------------------------ units

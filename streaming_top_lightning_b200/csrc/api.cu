@@ -8,8 +8,8 @@
 // list; the merge kernel folds them.  To keep the scratch bounded
 // independently of S, query tiles are processed in blocks sized so that one
 // block's partial lists fit the scratch budget: one score launch and one merge
-// launch per block.  With key_chunk = 0 a single chunk covers each query's
-// keys, units write the final answer directly and no merge pass runs.
+// launch per block; a row-sort launch orders the whole output at the end.
+// With key_chunk = 0 a single chunk covers each query's keys.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -106,34 +106,33 @@ int read_opts(const si_options* o, Opts* out) {
   return SI_OK;
 }
 
-// The plan of one problem: tiles, chunks and query blocks.
+// The plan of one problem: tiles, chunks and query blocks.  Every (tile,
+// chunk) unit leaves an L-key partial list per query; the query tiles of one
+// launch block share a scratch of B * tb * nch_max * QT * L keys, sized to the
+// scratch budget, so the scratch does not grow with S.
 struct Plan {
-  int QT, G, T, C, nch_max, tb, n_blocks;
+  int QT, G, T, C, nch_max, L, tb, n_blocks;
   size_t counters_bytes, partial_bytes;
   size_t ws_bytes() const { return align256(counters_bytes) + partial_bytes; }
 };
 
-Plan make_plan(int B, int S, int m, int K, int QT, const Opts& o) {
+Plan make_plan(int B, int S, int T, int K, int QT, const Opts& o) {
   Plan p{};
   p.QT = QT;
-  p.T = S / m;
+  p.T = T;
   p.G = (S + QT - 1) / QT;
-  const int tround = ((p.T > 0 ? p.T : 1) + 127) / 128 * 128;
+  const int tround = ((T > 0 ? T : 1) + 127) / 128 * 128;
   p.C = o.key_chunk > 0 ? o.key_chunk : tround;
-  p.nch_max = p.T > 0 ? (p.T + p.C - 1) / p.C : 1;
-  if (p.nch_max <= 1) {
-    p.nch_max = 1;
-    p.tb = p.G;
-    p.partial_bytes = 0;
-  } else {
-    const size_t per_tile = (size_t)B * p.nch_max * QT * K * sizeof(uint64_t);
-    const size_t budget = (size_t)o.scratch_mb << 20;
-    size_t tb = budget / per_tile;
-    if (tb < 1) tb = 1;
-    if (tb > (size_t)p.G) tb = p.G;
-    p.tb = (int)tb;
-    p.partial_bytes = per_tile * p.tb;
-  }
+  p.nch_max = T > 0 ? (T + p.C - 1) / p.C : 1;
+  if (p.nch_max < 1) p.nch_max = 1;
+  p.L = partial_len(K);
+  const size_t per_tile = (size_t)B * p.nch_max * QT * p.L * sizeof(uint64_t);
+  const size_t budget = (size_t)o.scratch_mb << 20;
+  size_t tb = budget / per_tile;
+  if (tb < 1) tb = 1;
+  if (tb > (size_t)p.G) tb = p.G;
+  p.tb = (int)tb;
+  p.partial_bytes = per_tile * p.tb;
   p.n_blocks = (p.G + p.tb - 1) / p.tb;
   p.counters_bytes = sizeof(int);  // one unit counter shared by every launch
   return p;
@@ -170,15 +169,13 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   if ((rc = dev_info(&dev))) return rc;
   const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem);
   if (!sp_plan.ok) return SI_ERR_DIM;
-  const Plan pl = make_plan(B, S, m, K, sp_plan.QT, o);
+  const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
   if (!aligned16(ws)) return SI_ERR_ALIGN;
 
   int* counters = static_cast<int*>(ws);
   uint64_t* partial =
-      pl.partial_bytes ? reinterpret_cast<uint64_t*>(static_cast<char*>(ws) +
-                                                     align256(pl.counters_bytes))
-                       : nullptr;
+      reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + align256(pl.counters_bytes));
   if (cudaMemsetAsync(counters, 0, pl.counters_bytes, stream) != cudaSuccess) return SI_ERR_CUDA;
 
   const int esz = fp8 ? 1 : 2;
@@ -204,7 +201,8 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
     UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base};
     ScoreParams p{};
-    p.sel = SelParams{B, S, T, m, K, pl.QT, sp_plan.CS, sp_plan.cap, g_lo, n_tiles, pl.nch_max,
+    p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
+                      sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,
                       out_idx, out_score, partial};
     p.ug = ug;
     p.w = w;
@@ -222,8 +220,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     if (launch_score_topk(fp8, D, H, tm_q, tm_kc, p, grid, sp_plan.smem, stream) != cudaSuccess)
       return SI_ERR_CUDA;
     id_base += units + grid;
-    if (pl.nch_max > 1 && launch_merge(partial, p.sel, ug, stream) != cudaSuccess)
-      return SI_ERR_CUDA;
+    if (launch_merge(partial, p.sel, ug, stream) != cudaSuccess) return SI_ERR_CUDA;
   }
   // the selection leaves each row's K best unsorted; order them
   if (launch_sort_rows(out_idx, out_score, (int64_t)B * S, K, dev->sms, stream) != cudaSuccess)
@@ -239,7 +236,7 @@ int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_o
   Opts o;
   if ((rc = read_opts(opt, &o))) return rc;
   const int QT = 256 / H;
-  const Plan pl = make_plan(B, S, m, K, QT, o);
+  const Plan pl = make_plan(B, S, S / m, K, QT, o);
   *bytes = pl.ws_bytes();
   (void)fp8;
   return SI_OK;
@@ -357,38 +354,15 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   if ((rc = dev_info(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int QT = 4, CS = 1024;
-  const int cap = ((std::max(topk + 32, 2 * topk) + 31) / 32) * 32;
+  const int cap = ((std::max(topk + 64, 2 * topk) + 31) / 32) * 32;
   // the selection-only path sees T keys per row; m still sets visibility
-  Plan pl{};
-  {
-    pl.QT = QT;
-    pl.T = T;
-    pl.G = (S + QT - 1) / QT;
-    const int tround = (T + 127) / 128 * 128;
-    pl.C = o.key_chunk > 0 ? o.key_chunk : tround;
-    pl.nch_max = (T + pl.C - 1) / pl.C;
-    if (pl.nch_max <= 1) {
-      pl.nch_max = 1;
-      pl.tb = pl.G;
-      pl.partial_bytes = 0;
-    } else {
-      const size_t per_tile = (size_t)B * pl.nch_max * QT * topk * sizeof(uint64_t);
-      size_t tb = (((size_t)o.scratch_mb) << 20) / per_tile;
-      if (tb < 1) tb = 1;
-      if (tb > (size_t)pl.G) tb = pl.G;
-      pl.tb = (int)tb;
-      pl.partial_bytes = per_tile * pl.tb;
-    }
-    pl.n_blocks = (pl.G + pl.tb - 1) / pl.tb;
-    pl.counters_bytes = sizeof(int);
-  }
+  const Plan pl = make_plan(B, S, T, topk, QT, o);
   const size_t bytes = pl.ws_bytes();
   void* ws = nullptr;
   if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return SI_ERR_CUDA;
   int* counters = static_cast<int*>(ws);
-  uint64_t* partial = pl.partial_bytes ? reinterpret_cast<uint64_t*>(
-                                             static_cast<char*>(ws) + align256(pl.counters_bytes))
-                                       : nullptr;
+  uint64_t* partial =
+      reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + align256(pl.counters_bytes));
   rc = SI_OK;
   if (cudaMemsetAsync(counters, 0, pl.counters_bytes, st) != cudaSuccess) rc = SI_ERR_CUDA;
   int id_base = 0;
@@ -396,7 +370,8 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
     UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base};
-    SelParams sp{B, S, T, m, topk, QT, CS, cap, g_lo, n_tiles, pl.nch_max, out_idx, out_score,
+    SelParams sp{B,    S,       T,          m,       topk,    QT,     CS,
+                 cap,  pl.L,    g_lo,       n_tiles, pl.nch_max, out_idx, out_score,
                  partial};
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
@@ -405,7 +380,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     if (launch_topk_scores(scores, sp, ug, counters, dev->err,
                            (uint64_t)o.timeout_ms * 1000000ull, grid, st) != cudaSuccess)
       rc = SI_ERR_CUDA;
-    else if (pl.nch_max > 1 && launch_merge(partial, sp, ug, st) != cudaSuccess)
+    else if (launch_merge(partial, sp, ug, st) != cudaSuccess)
       rc = SI_ERR_CUDA;
     id_base += units + grid;
   }

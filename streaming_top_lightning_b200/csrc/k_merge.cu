@@ -2,12 +2,13 @@
 //
 // "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
 // Top-k", Abstract: a chunked partition-merge top-k driver keeps the indexer
-// from ever holding the full score tensor.  When a query's visible keys span
-// several key chunks, each chunk's unit leaves a sorted, 0-padded partial list
-// of its K best keys in scratch; this kernel folds them into the final answer.  Under
-// the strict total order of the 64-bit keys, the top K of a union equals the
-// top K of the per-part top Ks, so the result is exactly the top K over all
-// chunks.
+// from ever holding the full score tensor.  Each (query tile, key chunk) unit
+// leaves, per query, a 0-padded partial list of at most L candidate keys in
+// scratch, a superset of that chunk's K best.  This kernel folds a query's
+// lists and takes the exact K best.  Under the strict total order of the
+// 64-bit keys, the top K of a union equals the top K of the union of any
+// per-part supersets of the per-part top Ks, so the result is exactly the top
+// K over all chunks.
 //
 // One warp per query, with the same candidate pool, threshold and radix
 // select as the score kernel's selection (si_select.cuh); the result is
@@ -24,27 +25,23 @@ constexpr int kMergeWarps = 4;
 SI_DEV void pool_take_keys(const uint64_t* keys, int n, uint64_t* pool, int cap, int K, int& np,
                            uint64_t& theta, uint32_t* hist, int lane) {
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r0 = 0; r0 < n; r0 += 32) {
-    const int r = r0 + lane;
-    const uint64_t key = r < n ? keys[r] : 0ull;
-    bool take = key > theta;
-    uint32_t mask = __ballot_sync(0xFFFFFFFFu, take);
-    if (mask == 0u) continue;
-    int cnt = __popc(mask);
-    if (np + cnt > cap) {
+  for (int r0 = 0; r0 < n; r0 += 64) {
+    if (np + 64 > cap) {
       __syncwarp();
-      uint64_t th = theta;
-      if (!pool_prune(pool, &np, K, &th, lane) || np + 32 > cap) {
-        th = pool_shrink(pool, np, K, hist, lane);
+      if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
+        theta = pool_shrink(pool, np, K, hist, lane);
         np = K;
       }
-      theta = th;
-      take = take && key > theta;
-      mask = __ballot_sync(0xFFFFFFFFu, take);
-      cnt = __popc(mask);
     }
-    if (take) pool[np + __popc(mask & lt_mask)] = key;
-    np += cnt;
+    const int ra = r0 + lane, rb = r0 + 32 + lane;
+    const uint64_t ka = ra < n ? keys[ra] : 0ull;
+    const uint64_t kb = rb < n ? keys[rb] : 0ull;
+    const bool ta = ka > theta, tb = kb > theta;  // 0 (padding) never beats theta
+    const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta), mb = __ballot_sync(0xFFFFFFFFu, tb);
+    const int na = __popc(ma);
+    if (ta) pool[np + __popc(ma & lt_mask)] = ka;
+    if (tb) pool[np + na + __popc(mb & lt_mask)] = kb;
+    np += na + __popc(mb);
   }
   __syncwarp();
 }
@@ -66,14 +63,22 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   const int t = g * QT + qi;
   if (t >= sp.S) return;
   const int nch = tile_chunks(ug, g);
-  if (nch <= 1) return;
-
-  const uint64_t* base = partial + (((int64_t)b * sp.n_tiles + gl) * sp.nch_max) * QT * K;
+  const int L = sp.L;
+  const uint64_t* base = partial + (((int64_t)b * sp.n_tiles + gl) * sp.nch_max) * QT * L;
   int np = 0;
   uint64_t theta = 0ull;
   for (int c = 0; c < nch; ++c)
-    pool_take_keys(base + ((int64_t)c * QT + qi) * K, K, pool, cap, K, np, theta, hist, lane);
-  const int n = pool_finish(pool, np, K, hist, lane);
+    pool_take_keys(base + ((int64_t)c * QT + qi) * L, L, pool, cap, K, np, theta, hist, lane);
+  // exact K best: prune while far above K, then the radix select
+  __syncwarp();
+  if (np > K) {
+    uint64_t th;
+    while (np > K + K / 4 + 64 && pool_prune(pool, &np, K, &th, lane)) {
+    }
+    pool_shrink(pool, np, K, hist, lane);
+    np = K;
+  }
+  const int n = np;
   const int64_t o = ((int64_t)b * sp.S + t) * K;
   for (int r = lane; r < K; r += 32) {
     const bool real = r < n;
@@ -85,10 +90,10 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
 
 cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                          cudaStream_t stream) {
-  // pool room: twice K keeps radix selects rare, and at least one block of
-  // 32 beyond K
+  // pool room: twice K keeps radix selects rare, and at least one step of
+  // 64 keys beyond K
   const int K = sp.K;
-  const int cap = ((std::max(K + 32, 2 * K) + 31) / 32) * 32;
+  const int cap = ((std::max(K + 64, 2 * K) + 31) / 32) * 32;
   const size_t smem = sizeof(uint32_t) * kMergeWarps * 256 + sizeof(uint64_t) * kMergeWarps * cap;
   cudaError_t e =
       cudaFuncSetAttribute(k_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -37,7 +37,7 @@ constexpr int kEpiWarp0 = 2;    // first epilogue warp
 constexpr int kSelWarp0 = 6;    // first selection warp
 
 struct UnitInfo {
-  int valid, b, g, c, kbeg, kend, ntiles, direct;
+  int valid, b, g, c, kbeg, kend, ntiles;
 };
 
 struct ScoreCtlSmem {
@@ -174,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool ok = unit_decode(p.ug, id, b, g, c);
         const int r = ring_it % kRing;
         if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl)) break;
-        UnitInfo u{0, 0, 0, 0, 0, 0, 0, 0};
+        UnitInfo u{0, 0, 0, 0, 0, 0, 0};
         if (ok) {
           const int vmax = tile_vmax(p.ug, g);
           u.valid = 1;
@@ -184,7 +184,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           u.kbeg = c * p.ug.C;
           u.kend = min(u.kbeg + p.ug.C, vmax);
           u.ntiles = u.kend > u.kbeg ? (u.kend - u.kbeg + kM - 1) / kM : 0;
-          u.direct = tile_chunks(p.ug, g) == 1;
         }
         cs->ring[r] = u;
         mbar_arrive(smem_u32(&cs->unit_full[r]));
@@ -389,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pos >= CS || last) {
           if (ew == 0 && lane == 0) {
             const int nk = max(0, min(CS, u.kend - j_strip));
-            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0, u.direct};
+            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0};
           }
           mbar_arrive(smem_u32(&cs->strip_full[slot]));
           ++strip_it;
@@ -465,7 +464,7 @@ ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
   const size_t kc_bytes = (size_t)kM * D * esz;
   const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * 4 * kN +
                        sizeof(ScoreCtlSmem);
-  const int cap_min = ((std::max(K + 32, 64) + 31) / 32) * 32;
+  const int cap_min = ((K + 64 + 31) / 32) * 32;
   const int cap_max = ((2 * K + 31) / 32) * 32 > cap_min ? ((2 * K + 31) / 32) * 32 : cap_min;
   const int cs_max = std::min(1024, std::max(128, 4096 / QT));
   long best_score[5] = {-1, -1, -1, -1, -1};

@@ -79,7 +79,6 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
       const int vmax = tile_vmax(ug, g);
       const int kbeg = c * ug.C;
       const int kend = min(kbeg + ug.C, vmax);
-      const int direct = tile_chunks(ug, g) == 1;
       for (int j0 = kbeg;; j0 += CS) {
         const int nk = max(0, min(CS, kend - j0));
         const int last = (j0 + CS >= kend) ? 1 : 0;
@@ -99,7 +98,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
           const float* src = X + ((int64_t)b * sp.S + t) * sp.T + j0;
           for (int q = tid; q < lim; q += kLoadThreads) st[(size_t)qi * CS + q] = __ldg(src + q);
         }
-        if (tid == 0) meta[slot] = StripMeta{1, b, g, c, j0, nk, last, direct};
+        if (tid == 0) meta[slot] = StripMeta{1, b, g, c, j0, nk, last};
         mbar_arrive(full_bar + 8 * slot);
         ++it;
         if (last) break;

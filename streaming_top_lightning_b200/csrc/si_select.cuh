@@ -11,9 +11,10 @@
 // enters the pool only if it beats theta.  When the pool is full, a warp radix
 // select finds the exact K-th largest pool key, which becomes theta, and the
 // pool is compacted to the K keys at or above it.  A unit (a tile of QT
-// queries x one key chunk) ends with one last select; the K survivors are
-// written out unsorted, either as the final answer or as a partial list for
-// the merge kernel, and a separate pass (k_sort_rows.cu) orders the rows.
+// queries x one key chunk) ends by pruning its pool to at most L candidates,
+// written to scratch as the unit's partial list; the merge kernel
+// (k_merge.cu) takes the exact top K over a query's partial lists and the
+// row sort (k_sort_rows.cu) orders the result.
 // Every pass reads the pool with consecutive lanes on consecutive keys, so no
 // access has bank conflicts.
 #pragma once
@@ -31,18 +32,23 @@ struct StripMeta {
   int j0;      // first key of the strip
   int nkeys;   // keys in the strip (<= CS)
   int last;    // 1 if this is the unit's last strip
-  int direct;  // 1: the unit covers every visible key, write the final answer
 };
 
 struct SelParams {
   int B, S, T, m, K, QT, CS;
-  int cap;             // pool entries per query (>= K + 32)
+  int cap;             // pool entries per query (>= K + 64)
+  int L;               // length of a partial list (> K), see partial_len()
   int g_lo, n_tiles;   // query tiles [g_lo, g_lo + n_tiles) in this launch
   int nch_max;         // chunk slots per query tile in the partial scratch
   int32_t* out_idx;    // [B,S,K]
   float* out_score;    // [B,S,K]
-  uint64_t* partial;   // [B, n_tiles, nch_max, QT, K] selected keys, 0-padded
+  uint64_t* partial;   // [B, n_tiles, nch_max, QT, L] candidate keys, 0-padded
 };
+
+// A unit leaves at most this many candidates per query (a superset of its K
+// best): enough slack above K that pruning rarely has to fall back to the
+// exact select.
+__host__ __device__ constexpr int partial_len(int K) { return ((K + K / 4 + 64 + 31) / 32) * 32; }
 
 struct SelSmem {
   uint64_t* pool;      // [QT][cap] candidate keys
@@ -248,41 +254,25 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
   uint64_t theta = *th_p;
   int np = *np_p;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int p0 = 0; p0 < lim; p0 += 128) {
-    // four independent groups of 32 keys per round
-    uint64_t key[4];
-    bool take[4];
-    uint32_t mask[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int p = p0 + 32 * u + lane;
-      key[u] = p < lim ? make_key(st[p], j0 + p) : 0ull;
-      take[u] = p < lim && key[u] > theta;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) mask[u] = __ballot_sync(0xFFFFFFFFu, take[u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (mask[u] == 0u) continue;
-      int cnt = __popc(mask[u]);
-      if (np + cnt > cap) {
-        __syncwarp();
-        uint64_t th = theta;
-        if (!pool_prune(pool, &np, K, &th, lane) || np + 32 > cap) {
-          th = pool_shrink(pool, np, K, hist, lane);
-          np = K;
-        }
-        theta = th;
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          take[v] = take[v] && key[v] > theta;
-          mask[v] = __ballot_sync(0xFFFFFFFFu, take[v]);
-        }
-        cnt = __popc(mask[u]);
+  for (int p0 = 0; p0 < lim; p0 += 64) {
+    // room for this step's up to 64 keys; else raise theta first
+    if (np + 64 > cap) {
+      __syncwarp();
+      if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
+        theta = pool_shrink(pool, np, K, hist, lane);
+        np = K;
       }
-      if (take[u]) pool[np + __popc(mask[u] & lt_mask)] = key[u];
-      np += cnt;
     }
+    const int pa = p0 + lane, pb = p0 + 32 + lane;
+    const bool va = pa < lim, vb = pb < lim;
+    const uint64_t ka = va ? make_key(st[pa], j0 + pa) : 0ull;
+    const uint64_t kb = vb ? make_key(st[pb], j0 + pb) : 0ull;
+    const bool ta = va && ka > theta, tb = vb && kb > theta;
+    const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta), mb = __ballot_sync(0xFFFFFFFFu, tb);
+    const int na = __popc(ma);
+    if (ta) pool[np + __popc(ma & lt_mask)] = ka;
+    if (tb) pool[np + na + __popc(mb & lt_mask)] = kb;
+    np += na + __popc(mb);
   }
   __syncwarp();
   if (lane == 0) {
@@ -292,40 +282,29 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
   __syncwarp();
 }
 
-// Final select of a query's pool: afterwards pool[0, n) holds its n = min(np, K)
-// best keys, in no particular order (the output rows are sorted afterwards by
-// a separate pass over the result).
-SI_DEV int pool_finish(uint64_t* pool, int np, int K, uint32_t* hist, int lane) {
+// End of a unit: prune the pool until it fits a partial list of L keys (a
+// superset of the K best; the exact selection happens in the merge kernel).
+// Returns the number of keys left in pool[0, n).
+SI_DEV int pool_trim(uint64_t* pool, int np, int K, int L, uint32_t* hist, int lane) {
   __syncwarp();
-  if (np > K) {
-    uint64_t th;
-    while (np > K + K / 4 + 64 && pool_prune(pool, &np, K, &th, lane)) {
+  uint64_t th;
+  while (np > L) {
+    if (!pool_prune(pool, &np, K, &th, lane)) {
+      pool_shrink(pool, np, K, hist, lane);
+      np = K;
     }
-    pool_shrink(pool, np, K, hist, lane);
-    np = K;
   }
   __syncwarp();
   return np;
 }
 
-// Write one query's selected keys out (final answer or partial list), unsorted.
+// Write one query's candidates out as its partial list for (tile, chunk).
 SI_DEV void warp_emit(const SelParams& p, const StripMeta& md, int qi, const uint64_t* keys,
                       int n, int lane) {
-  const int t = md.g * p.QT + qi;
-  if (md.direct) {
-    const int64_t base = ((int64_t)md.b * p.S + t) * p.K;
-    for (int r = lane; r < p.K; r += 32) {
-      const bool real = r < n;
-      const uint64_t k = real ? keys[r] : 0ull;
-      p.out_idx[base + r] = real ? key_index(k) : -1;
-      p.out_score[base + r] = real ? key_score(k) : __int_as_float(0xFF800000);
-    }
-  } else {
-    const int64_t slot =
-        (((int64_t)md.b * p.n_tiles + (md.g - p.g_lo)) * p.nch_max + md.c) * p.QT + qi;
-    uint64_t* dst = p.partial + slot * p.K;
-    for (int r = lane; r < p.K; r += 32) dst[r] = r < n ? keys[r] : 0ull;
-  }
+  const int64_t slot =
+      (((int64_t)md.b * p.n_tiles + (md.g - p.g_lo)) * p.nch_max + md.c) * p.QT + qi;
+  uint64_t* dst = p.partial + slot * p.L;
+  for (int r = lane; r < p.L; r += 32) dst[r] = r < n ? keys[r] : 0ull;
   __syncwarp();
 }
 
@@ -349,7 +328,7 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
       pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), pool,
                       p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane);
       if (md.last) {
-        const int n = pool_finish(pool, sm.npool[qi], p.K, hist, lane);
+        const int n = pool_trim(pool, sm.npool[qi], p.K, p.L, hist, lane);
         warp_emit(p, md, qi, pool, n, lane);
         if (lane == 0) {
           sm.npool[qi] = 0;

@@ -222,8 +222,9 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     id_base += units + grid;
     if (launch_merge(partial, p.sel, ug, stream) != cudaSuccess) return SI_ERR_CUDA;
   }
-  // the selection leaves each row's K best unsorted; order them
-  if (launch_sort_rows(out_idx, out_score, (int64_t)B * S, K, dev->sms, stream) != cudaSuccess)
+  // rows of more than 512 keys leave the merge unsorted; order them
+  if (!merge_sorts_rows(K) &&
+      launch_sort_rows(out_idx, out_score, (int64_t)B * S, K, dev->sms, stream) != cudaSuccess)
     return SI_ERR_CUDA;
   return SI_OK;
 }
@@ -384,7 +385,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
       rc = SI_ERR_CUDA;
     id_base += units + grid;
   }
-  if (rc == SI_OK &&
+  if (rc == SI_OK && !merge_sorts_rows(topk) &&
       launch_sort_rows(out_idx, out_score, (int64_t)B * S, topk, dev->sms, st) != cudaSuccess)
     rc = SI_ERR_CUDA;
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;

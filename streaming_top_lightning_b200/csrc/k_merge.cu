@@ -11,8 +11,9 @@
 // K over all chunks.
 //
 // One warp per query, with the same candidate pool, threshold and radix
-// select as the score kernel's selection (si_select.cuh); the result is
-// written unsorted, like the score kernel's, for the row sort that follows.
+// select as the score kernel's selection (si_select.cuh).  For K <= 512 the
+// warp also sorts its row in registers; larger rows are written unsorted and
+// ordered by the row-sort kernel.
 #include <algorithm>
 
 #include "si_kernels.h"
@@ -44,6 +45,77 @@ SI_DEV void pool_take_keys(const uint64_t* keys, int n, uint64_t* pool, int cap,
     np += na + __popc(mb);
   }
   __syncwarp();
+}
+
+// Bitonic sort of 32*R keys held by one warp, blocked layout: lane l holds
+// elements l*R .. l*R+R-1 in v[0..R).  Distances below R pair registers of one
+// lane; larger ones pair lanes through xor-shuffles.  The lower index of each
+// pair keeps the max where (index & size) == 0, so the result is descending.
+template <int R, int S>
+SI_DEV void bsort_reg(uint64_t (&v)[R], int lane, int size) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if ((r & S) == 0) {
+      const bool dir = ((lane * R + r) & size) == 0;
+      const uint64_t a = v[r], b = v[r | S];
+      const bool gt = a > b;
+      const uint64_t mx = gt ? a : b, mn = gt ? b : a;
+      v[r] = dir ? mx : mn;
+      v[r | S] = dir ? mn : mx;
+    }
+  }
+}
+
+template <int R>
+SI_DEV void warp_sort_blocked(uint64_t (&v)[R], int lane) {
+#pragma unroll 1
+  for (int size = 2; size <= 32 * R; size <<= 1) {
+#pragma unroll 1
+    for (int s = size >> 1; s > 0; s >>= 1) {
+      if (s >= R) {
+        const int lm = s / R;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool dir = ((lane * R + r) & size) == 0;
+          const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, v[r], lm);
+          const bool gt = v[r] > y;
+          v[r] = ((lower == dir) == gt) ? v[r] : y;
+        }
+      } else if (s == 8) {
+        if constexpr (R > 8) bsort_reg<R, 8>(v, lane, size);
+      } else if (s == 4) {
+        if constexpr (R > 4) bsort_reg<R, 4>(v, lane, size);
+      } else if (s == 2) {
+        if constexpr (R > 2) bsort_reg<R, 2>(v, lane, size);
+      } else {
+        if constexpr (R > 1) bsort_reg<R, 1>(v, lane, size);
+      }
+    }
+  }
+}
+
+// Sort the n (<= 32*R) selected keys in pool[0, n) and write the row.  The
+// pool is unsorted, so reading it lane-interleaved (conflict-free) and
+// treating that as the blocked layout loses nothing.
+template <int R>
+SI_DEV void sort_and_write(const uint64_t* pool, int n, int K, int32_t* oi, float* os, int lane) {
+  uint64_t v[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int i = 32 * r + lane;
+    v[r] = i < n ? pool[i] : 0ull;
+  }
+  warp_sort_blocked<R>(v, lane);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = lane * R + r;
+    if (e < K) {
+      const uint64_t k = v[r];
+      oi[e] = k ? key_index(k) : -1;
+      os[e] = k ? key_score(k) : __int_as_float(0xFF800000);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kMergeWarps * 32)
@@ -80,6 +152,18 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   }
   const int n = np;
   const int64_t o = ((int64_t)b * sp.S + t) * K;
+  __syncwarp();
+  // K <= 512: sort here, in registers; larger K: unsorted rows, ordered by
+  // the row-sort kernel afterwards
+  const int n2 = pow2ceil(K < 32 ? 32 : K);
+  switch (n2) {
+    case 32: return sort_and_write<1>(pool, n, K, sp.out_idx + o, sp.out_score + o, lane);
+    case 64: return sort_and_write<2>(pool, n, K, sp.out_idx + o, sp.out_score + o, lane);
+    case 128: return sort_and_write<4>(pool, n, K, sp.out_idx + o, sp.out_score + o, lane);
+    case 256: return sort_and_write<8>(pool, n, K, sp.out_idx + o, sp.out_score + o, lane);
+    case 512: return sort_and_write<16>(pool, n, K, sp.out_idx + o, sp.out_score + o, lane);
+    default: break;
+  }
   for (int r = lane; r < K; r += 32) {
     const bool real = r < n;
     const uint64_t k = real ? pool[r] : 0ull;
@@ -87,6 +171,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
     sp.out_score[o + r] = real ? key_score(k) : __int_as_float(0xFF800000);
   }
 }
+
+bool merge_sorts_rows(int K) { return K <= 512; }
 
 cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                          cudaStream_t stream) {

@@ -47,6 +47,9 @@ cudaError_t launch_topk_scores(const float* X, const SelParams& sp, const UnitGr
 cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                          cudaStream_t stream);
 
+// True when the merge kernel already writes sorted rows (small K).
+bool merge_sorts_rows(int K);
+
 // Sorts each of the rows [rows, K] of (idx, score) in place into the output
 // order (score descending, index ascending, padding last).
 cudaError_t launch_sort_rows(int32_t* idx, float* score, int64_t rows, int K, int sms,

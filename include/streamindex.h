@@ -131,6 +131,33 @@ int si_quantize_fp8_rows(const void* x, int64_t rows, int cols, void* x8, float*
 int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, int32_t* out_idx,
                    float* out_score, const si_options* opt, void* stream);
 
+/*
+ * si_indexer_topk_noalloc: si_indexer_topk for callers that cannot allocate
+ * device memory.  The StreamIndex paper has no counterpart; this entry point
+ * exists for callers embedded in a runtime that owns every device allocation
+ * (a serving engine with a fixed memory pool, a plugin inside another
+ * framework) or that cannot afford an allocator call in a latency-critical
+ * loop, where an allocation may block on the allocator or fail when memory is
+ * fragmented.
+ *   Arguments, layouts and results are those of si_indexer_topk.  The call
+ *   makes no cudaMalloc, cudaMallocAsync or cudaFree: its scratch is a fixed
+ *   64 MiB device array inside the library (SI_NOALLOC_SCRATCH_BYTES), which
+ *   every GPU that loads the library holds until the process exits.  Query
+ *   tiles are processed in blocks sized to that array; a problem whose single
+ *   query tile needs more than it returns SI_ERR_WORKSPACE.
+ *   The first call on each device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.
+ *   All calls share the one array and each leaves its contents behind; the
+ *   call clears what must start at zero (its work counter) on `stream` before
+ *   use.  Calls whose work overlaps on the GPU (different streams, or other
+ *   threads) race on the array and give undefined results: serialise them.
+ */
+#define SI_NOALLOC_SCRATCH_BYTES (64u << 20)
+int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                            int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                            void* stream);
+
 /* ---- diagnostics ------------------------------------------------------ */
 
 /* Text for a status code (static storage). */

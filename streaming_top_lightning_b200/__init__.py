@@ -19,7 +19,7 @@ from . import _lib
 from ._lib import SiOptions, StreamIndexError  # noqa: F401
 
 __all__ = [
-    "indexer_topk", "indexer_topk_fp8", "quantize_fp8_rows", "topk_scores", "workspace_size",
+    "indexer_topk", "indexer_topk_noalloc", "indexer_topk_fp8", "quantize_fp8_rows", "topk_scores", "workspace_size",
     "device_error", "options", "version", "StreamIndexError",
 ]
 
@@ -105,6 +105,23 @@ def indexer_topk(q, w, kc, m: int, topk: int, *, out=None, opts: SiOptions | Non
                                 _ptr(score), ctypes.byref(opts) if opts else None,
                                 _ptr(workspace), workspace.numel(), st)
     _lib.check("si_indexer_topk_ex", rc)
+    return idx, score
+
+
+def indexer_topk_noalloc(q, w, kc, m: int, topk: int, *, out=None, stream=None):
+    """``indexer_topk`` through the entry point that allocates no device memory
+    (its scratch is a fixed array inside the library; see
+    si_indexer_topk_noalloc in include/streamindex.h).  Returns (idx, score);
+    pass ``out`` to avoid allocating the outputs here as well."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    _need(w, torch.float32, 3, "w")
+    _need(kc, torch.bfloat16, 3, "kc")
+    B, S, H, D = q.shape
+    idx, score = _outputs(B, S, topk, q.device, out)
+    rc = _lib.load().si_indexer_topk_noalloc(_ptr(q), _ptr(w), _ptr(kc), B, S, H, D, m, topk,
+                                             _ptr(idx), _ptr(score), _stream(stream))
+    _lib.check("si_indexer_topk_noalloc", rc)
     return idx, score
 
 

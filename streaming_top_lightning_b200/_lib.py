@@ -22,7 +22,7 @@ STATUS = {
 EXPORTS = [
     "si_indexer_topk", "si_indexer_topk_workspace_size", "si_indexer_topk_ex",
     "si_indexer_topk_fp8", "si_quantize_fp8_rows", "si_topk_scores", "si_status_string",
-    "si_get_last_device_error", "si_version",
+    "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc",
 ]
 
 
@@ -52,6 +52,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     P, I, L, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     OP = ctypes.POINTER(SiOptions)
     lib.si_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P]
+    lib.si_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P]
     lib.si_indexer_topk_workspace_size.argtypes = [I, I, I, I, I, I, OP, ctypes.POINTER(Z)]
     lib.si_indexer_topk_ex.argtypes = [P, P, P, I, I, I, I, I, I, P, P, OP, P, Z, P]
     lib.si_indexer_topk_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, OP, P, Z, P]

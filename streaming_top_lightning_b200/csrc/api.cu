@@ -243,6 +243,31 @@ int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_o
   return SI_OK;
 }
 
+// ------------------------------------------------------------ fixed scratch
+// Device scratch for si_indexer_topk_noalloc: a file-scope array, so the call
+// needs no allocation.  Every GPU that loads the library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the fixed scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SI_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SI_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SI_OK;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------ unit counting
@@ -400,6 +425,23 @@ int si_get_last_device_error(void* stream) {
   if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof zero) != cudaSuccess) return SI_ERR_CUDA;
   if (v & SI_DEVERR_TIMEOUT) return SI_ERR_DEVICE_TIMEOUT;
   return v ? SI_ERR_CUDA : SI_OK;
+}
+
+int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                            int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                            void* stream) {
+  int rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score);
+  if (rc) return rc;
+  // query blocks sized to the fixed scratch (its last MiB left for the counter)
+  si_options opt{};
+  opt.scratch_mb = (int)(kNoAllocScratchBytes >> 20) - 1;
+  size_t need = 0;
+  if ((rc = workspace_for(false, S, B, H_I, d_I, m, topk, &opt, &need))) return rc;
+  if (need > kNoAllocScratchBytes) return SI_ERR_WORKSPACE;  // one query tile does not fit
+  void* ws = nullptr;
+  if ((rc = noalloc_scratch(&ws))) return rc;
+  return run_indexer(false, q, nullptr, w, kc, nullptr, B, S, H_I, d_I, m, topk, out_idx,
+                     out_score, &opt, ws, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -198,6 +198,24 @@ def run_reference(args, sh):
     return 0
 
 
+def kernel_launches_per_step(sh, args) -> int:
+    """Our kernel launches in one step: a score and a merge launch per query
+    block, the row sort when topk > 512, and the two quantiser launches of the
+    FP8 path.  The query-block count follows the library's scratch plan (512 MiB
+    of partial lists by default; 256/H_I queries per tile; partial lists of
+    ceil((K + K/4 + 64)/32)*32 keys per query and key chunk)."""
+    QT = 256 // sh.H
+    G = (sh.S + QT - 1) // QT
+    C = args.key_chunk if args.key_chunk else (sh.T + 127) // 128 * 128
+    nch = max(1, (sh.T + C - 1) // C)
+    L = (sh.topk + sh.topk // 4 + 64 + 31) // 32 * 32
+    per_tile = sh.B * nch * QT * L * 8
+    tb = max(1, min(G, (512 << 20) // per_tile))
+    n_blocks = (G + tb - 1) // tb
+    n = 2 * n_blocks + (1 if sh.topk > 512 else 0)
+    return n + (2 if args.fp8 else 0)
+
+
 def config_of(sh, args):
     return {"workload": sh.name, "B": sh.B, "S": sh.S, "T": sh.T, "m": sh.m, "H_I": sh.H,
             "d_I": sh.D, "topk": sh.topk, "key_chunk": args.key_chunk,
@@ -254,6 +272,11 @@ def run_native(args, sh):
     w_d = w_h.to(dev)
     kc_d = kc_h.to(dev).view(torch.bfloat16)
     opts = stl.options(key_chunk=args.key_chunk)
+    timed = {"opts": None}
+
+    def step_opts():
+        # inside the timed region each step records its score-kernel events
+        return opts if timed["opts"] is None else timed["opts"]
     ws = torch.empty(max(16, stl.workspace_size(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, opts)),
                      dtype=torch.uint8, device=dev)
     idx = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32, device=dev)
@@ -264,10 +287,10 @@ def run_native(args, sh):
             a8, s_q = stl.quantize_fp8_rows(q_d)
             b8, s_k = stl.quantize_fp8_rows(kc_d)
             stl.indexer_topk_fp8(a8, s_q, w_d, b8, s_k, sh.m, sh.topk, out=(idx, score),
-                                 opts=opts, workspace=ws)
+                                 opts=step_opts(), workspace=ws)
     else:
         def step():
-            stl.indexer_topk(q_d, w_d, kc_d, sh.m, sh.topk, out=(idx, score), opts=opts,
+            stl.indexer_topk(q_d, w_d, kc_d, sh.m, sh.topk, out=(idx, score), opts=step_opts(),
                              workspace=ws)
 
     stream = torch.cuda.current_stream()
@@ -291,15 +314,25 @@ def run_native(args, sh):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
+    # the library records the score kernel's own launch interval into these
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for a, b in kev:  # make sure the events exist before their handles are taken
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    kopts = [stl.options(key_chunk=args.key_chunk, score_events=e) for e in kev]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
         barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
         for i in range(K):
+            timed["opts"] = kopts[i]
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
+        timed["opts"] = None
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -307,7 +340,8 @@ def run_native(args, sh):
     if rc != 0:
         raise RuntimeError(f"device error {rc} in the timed region")
     total_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
 
     # end to end through the public API: host -> device inputs, the call,
     # device -> host result, every step
@@ -366,11 +400,7 @@ def finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2
     peak_tf = float(peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
     tflops_step = flops_launch / (ms_per_step / 1e3) / 1e12
     traffic = traffic_record(sh.name, args.fp8)
-    # our kernels per step: the score kernel per query block (+ the merge kernel
-    # when keys are chunked), plus the two quantiser launches on the FP8 path
-    launches_per_step = 1 + (1 if args.key_chunk and args.key_chunk < sh.T else 0)
-    if args.fp8:
-        launches_per_step += 2
+    launches_per_step = kernel_launches_per_step(sh, args)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

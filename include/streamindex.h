@@ -69,6 +69,14 @@ typedef struct si_options {
   int debug_flags;      /* bit 0: the producer never issues its first load, so
                            the first consumer wait must expire (tests the
                            timeout path).  Default 0. */
+  void* score_events[2];/* optional cudaEvent_t pair (NULL = none): the call
+                           records [0] on `stream` just before its first
+                           score-kernel launch and [1] just after its last
+                           one, so cudaEventElapsedTime gives the fused score
+                           kernel's own device time.  With several query
+                           blocks, the merge launches between them fall
+                           inside the interval.  The events stay owned by
+                           the caller. */
 } si_options;
 
 /* ---- the indexer step ------------------------------------------------ */

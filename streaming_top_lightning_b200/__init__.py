@@ -51,8 +51,16 @@ def _need(t, dtype, ndim, name):
 
 
 def options(key_chunk: int = 0, scratch_mb: int = 0, grid_ctas: int = 0, timeout_ms: int = 0,
-            debug_flags: int = 0) -> SiOptions:
-    return SiOptions(key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags)
+            debug_flags: int = 0, score_events=None) -> SiOptions:
+    """Tuning knobs of include/streamindex.h.  ``score_events`` is an optional
+    pair of ``torch.cuda.Event(enable_timing=True)`` that the call records around
+    its score-kernel launches (on the call's stream)."""
+    o = SiOptions(key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags)
+    if score_events is not None:
+        a, b = score_events
+        o.score_events[0] = a.cuda_event
+        o.score_events[1] = b.cuda_event
+    return o
 
 
 def version() -> int:

@@ -29,7 +29,7 @@ EXPORTS = [
 class SiOptions(ctypes.Structure):
     _fields_ = [("key_chunk", ctypes.c_int), ("scratch_mb", ctypes.c_int),
                 ("grid_ctas", ctypes.c_int), ("timeout_ms", ctypes.c_int),
-                ("debug_flags", ctypes.c_int)]
+                ("debug_flags", ctypes.c_int), ("score_events", ctypes.c_void_p * 2)]
 
 
 class StreamIndexError(RuntimeError):

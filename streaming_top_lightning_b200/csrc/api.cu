@@ -89,11 +89,14 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t 
 
 struct Opts {
   int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags;
+  cudaEvent_t ev_begin, ev_end;
 };
 
 int read_opts(const si_options* o, Opts* out) {
-  Opts d{0, 512, 0, 2000, 0};
+  Opts d{0, 512, 0, 2000, 0, nullptr, nullptr};
   if (o) {
+    d.ev_begin = static_cast<cudaEvent_t>(o->score_events[0]);
+    d.ev_end = static_cast<cudaEvent_t>(o->score_events[1]);
     d.key_chunk = o->key_chunk;
     d.scratch_mb = o->scratch_mb > 0 ? o->scratch_mb : 512;
     d.grid_ctas = o->grid_ctas;
@@ -217,7 +220,11 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
     if (grid < 1) grid = 1;
+    if (blk == 0 && o.ev_begin && cudaEventRecord(o.ev_begin, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
     if (launch_score_topk(fp8, D, H, tm_q, tm_kc, p, grid, sp_plan.smem, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
+    if (blk + 1 == pl.n_blocks && o.ev_end && cudaEventRecord(o.ev_end, stream) != cudaSuccess)
       return SI_ERR_CUDA;
     id_base += units + grid;
     if (launch_merge(partial, p.sel, ug, stream) != cudaSuccess) return SI_ERR_CUDA;

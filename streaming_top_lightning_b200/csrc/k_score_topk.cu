@@ -12,15 +12,19 @@
 // epilogue thread reduces the heads of its own key without any cross-lane
 // traffic: one max and half a packed FMA per accumulator element.
 //
-// Warp roles (320 threads, one CTA per SM, persistent):
-//   warp 0     TMA producer and unit scheduler: takes (tile, chunk) units from
-//              a global counter, loads the query tile once per unit and streams
-//              128-key tiles of kc through an NST-stage mbarrier ring;
-//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma (one thread)
-//              into two 256-column accumulators used alternately;
-//   warps 2-5  epilogue: tcgen05.ld, ReLU, w-weighted head sum (x s_k for FP8),
-//              scores into a shared-memory strip; never to global memory;
-//   warps 6-9  streaming selection (si_select.cuh) on the strips.
+// Warp roles (448 threads, one CTA per SM, persistent):
+//   warp 0      TMA producer and unit scheduler: takes (tile, chunk) units from
+//               a global counter, loads the query tile once per unit and streams
+//               128-key tiles of kc through an NST-stage mbarrier ring;
+//   warp 1      allocates 512 TMEM columns and issues tcgen05.mma (one thread)
+//               into two 256-column accumulators used alternately;
+//   warps 2-9   epilogue: warp w reads TMEM lane quadrant w%4 (32 keys) and
+//               column half (w-2)/4 (128 columns: QT/2 queries); tcgen05.ld,
+//               ReLU, w-weighted head sum (x s_k for FP8) in several
+//               independent packed-FMA chains per query, scores into a
+//               shared-memory strip; never to global memory;
+//   warps 10-13 streaming selection (si_select.cuh) on the strips.
+// So every SM sub-partition runs two epilogue warps and one selection warp.
 // Every wait is bounded (si_common.cuh); on expiry the CTA drains its own
 // asynchronous copies and MMAs, frees TMEM and exits with an error word set.
 #include <algorithm>
@@ -29,12 +33,16 @@
 
 namespace si {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kRing = 4;        // unit ring depth
 constexpr int kN = 256;         // MMA N: query-tile rows (QT * H)
 constexpr int kM = 128;         // MMA M: keys per tile
 constexpr int kEpiWarp0 = 2;    // first epilogue warp
-constexpr int kSelWarp0 = 6;    // first selection warp
+constexpr int kEpiWarps = 8;    // two per TMEM lane quadrant, one per column half
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kHalfN = kN / 2;  // accumulator columns per epilogue warp
+constexpr int kSelWarp0 = kEpiWarp0 + kEpiWarps;  // first selection warp
+static_assert(kThreads == (kSelWarp0 + kSelWarps) * 32, "warp roles");
 
 struct UnitInfo {
   int valid, b, g, c, kbeg, kend, ntiles;
@@ -83,18 +91,33 @@ SI_DEV void tmem_ld_fence(float (&v)[32]) {
                  "+f"(v[30]), "+f"(v[31]));
 }
 
-// Weighted ReLU head sum of one 32-column chunk into the per-query packed
-// accumulators.  Column c of the chunk is query (ch*32 + c) / H, head
-// (ch*32 + c) % H; w2 holds the unit's weights as float2 pairs.
-template <int H, int QT>
-SI_DEV void epi_chunk(int ch, const float (&v)[32], const float2* w2, float2 (&acc)[QT]) {
+// Independent packed accumulators per query of an epilogue warp: enough
+// chains to cover the FMA latency, at most 8 float2 in all.
+template <int H>
+struct EpiGeom {
+  static constexpr int kQH = kHalfN / H;               // queries per column half
+  static constexpr int kNA = kQH >= 8 ? 1 : 8 / kQH;   // chains per query
+  static_assert(kQH * kNA <= 16 && (H / 2) % kNA == 0, "accumulator split");
+};
+
+// Weighted ReLU head sum of one 32-column chunk of this warp's column half
+// into the packed accumulators.  Local column c = ch*32 + e is query c / H of
+// the half and head c % H; head pair (c % H)/2 feeds chain ((c % H)/2) % kNA.
+// w4 holds the half's weights as float4 groups (one LDS.128 per 4 columns).
+template <int H>
+SI_DEV void epi_chunk(int ch, const float (&v)[32], const float4* w4,
+                      float2 (&acc)[EpiGeom<H>::kQH][EpiGeom<H>::kNA]) {
+  constexpr int NA = EpiGeom<H>::kNA;
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
+  for (int e = 0; e < 32; e += 4) {
     const int col = ch * 32 + e;
-    const int qi = col / H;
-    const float2 wv = w2[col >> 1];
-    const float2 r = make_float2(fmaxf(v[e], 0.0f), fmaxf(v[e + 1], 0.0f));
-    acc[qi] = __ffma2_rn(wv, r, acc[qi]);
+    const int ql = col / H;
+    const int a0 = ((col % H) >> 1) % NA, a1 = (((col + 2) % H) >> 1) % NA;
+    const float4 wv = w4[col >> 2];
+    const float2 r0 = make_float2(fmaxf(v[e], 0.0f), fmaxf(v[e + 1], 0.0f));
+    const float2 r1 = make_float2(fmaxf(v[e + 2], 0.0f), fmaxf(v[e + 3], 0.0f));
+    acc[ql][a0] = __ffma2_rn(make_float2(wv.x, wv.y), r0, acc[ql][a0]);
+    acc[ql][a1] = __ffma2_rn(make_float2(wv.z, wv.w), r1, acc[ql][a1]);
   }
 }
 
@@ -118,8 +141,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sel_base = reinterpret_cast<uint8_t*>(strip + 2 * QT * CS);
   SelSmem sm;
   sel_state_carve(sel_base, QT, sp.cap, sm);
-  float* w_s = reinterpret_cast<float*>(sel_base + sel_state_bytes(QT, sp.cap));  // [4][kN]
-  ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + 4 * kN);
+  // [kEpiWarps][kHalfN]: each epilogue warp's private copy of its half of the weights
+  float* w_s = reinterpret_cast<float*>(sel_base + sel_state_bytes(QT, sp.cap));
+  ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + kEpiWarps * kHalfN);
 
   const uint32_t q_addr = smem_u32(q_s), kc_addr = smem_u32(kc_s);
   if (tid == 0) {
@@ -129,15 +153,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&cs->acc_full[i]), 1);
-      mbar_init(smem_u32(&cs->acc_empty[i]), 128);
-      mbar_init(smem_u32(&cs->strip_full[i]), 128);
+      mbar_init(smem_u32(&cs->acc_empty[i]), kEpiThreads);
+      mbar_init(smem_u32(&cs->strip_full[i]), kEpiThreads);
       mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);
     }
     mbar_init(smem_u32(&cs->q_full), 1);
     mbar_init(smem_u32(&cs->q_empty), 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&cs->unit_full[i]), 1);
-      mbar_init(smem_u32(&cs->unit_empty[i]), 1 + 4);
+      mbar_init(smem_u32(&cs->unit_empty[i]), 1 + kEpiWarps);
     }
     mbar_init(smem_u32(&cs->drain), 1);
     cs->abort = 0u;
@@ -293,11 +317,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kSelWarp0) {
     // ---------------------------------------------------------- epilogue
-    const int ew = warp - kEpiWarp0;  // 0..3
+    using EG = EpiGeom<H>;
+    constexpr int QH = EG::kQH, NA = EG::kNA;
+    const int ew = warp - kEpiWarp0;  // 0..7
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;         // column half: queries [half*QH, half*QH + QH)
     const int kl = quad * 32 + lane;  // key within the tile
-    float* wq = w_s + ew * kN;        // this warp's private copy of the unit's weights
-    const float2* w2 = reinterpret_cast<const float2*>(wq);
+    float* wq = w_s + ew * kHalfN;    // this warp's private copy of its half's weights
+    const float4* w4 = reinterpret_cast<const float4*>(wq);
     uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
     for (;;) {
       const int r = ring_it % kRing;
@@ -318,12 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the unit's weights (FP8: folded with the query row scales, which are
       // positive, so relu(s*x) = s*relu(x))
       const int64_t wrow = (int64_t)u.b * sp.S + (int64_t)u.g * QT;
-      for (int i = lane; i < kN; i += 32) {
-        const int qi = i / H;
+      for (int i = lane; i < kHalfN; i += 32) {
+        const int col = half * kHalfN + i;  // column of the 256-wide tile
         float wv = 0.0f;
-        if (u.g * QT + qi < sp.S) {
-          wv = p.w[wrow * H + i];
-          if (FP8) wv *= p.s_q[wrow * H + i];
+        if (u.g * QT + col / H < sp.S) {
+          wv = p.w[wrow * H + col];
+          if (FP8) wv *= p.s_q[wrow * H + col];
         }
         wq[i] = wv;
       }
@@ -346,41 +373,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ab * kN;
-          float2 acc[QT];
+          const uint32_t taddr =
+              tmem + ((uint32_t)(quad * 32) << 16) + ab * kN + half * kHalfN;
+          float2 acc[QH][NA];
 #pragma unroll
-          for (int qi = 0; qi < QT; ++qi) acc[qi] = make_float2(0.0f, 0.0f);
+          for (int ql = 0; ql < QH; ++ql)
+#pragma unroll
+            for (int a = 0; a < NA; ++a) acc[ql][a] = make_float2(0.0f, 0.0f);
           float va[32], vb[32];
           tmem_ld32(taddr, va);
+          tmem_ld32(taddr + 32, vb);
           tmem_ld_wait();
           tmem_ld_fence(va);
-#pragma unroll
-          for (int ch = 0; ch < kN / 32; ch += 2) {
-            tmem_ld32(taddr + (ch + 1) * 32, vb);
-            epi_chunk<H, QT>(ch, va, w2, acc);
-            tmem_ld_wait();
-            tmem_ld_fence(vb);
-            if (ch + 2 < kN / 32) tmem_ld32(taddr + (ch + 2) * 32, va);
-            epi_chunk<H, QT>(ch + 1, vb, w2, acc);
-            if (ch + 2 < kN / 32) {
-              tmem_ld_wait();
-              tmem_ld_fence(va);
-            }
-          }
+          tmem_ld_fence(vb);
+          epi_chunk<H>(0, va, w4, acc);
+          tmem_ld32(taddr + 64, va);
+          epi_chunk<H>(1, vb, w4, acc);
+          tmem_ld32(taddr + 96, vb);
+          tmem_ld_wait();
+          tmem_ld_fence(va);
+          tmem_ld_fence(vb);
+          // every column of this accumulator is in registers: release it
           tc_fence_before();
           mbar_arrive(smem_u32(&cs->acc_empty[ab]));
           ++acc_it;
+          epi_chunk<H>(2, va, w4, acc);
+          epi_chunk<H>(3, vb, w4, acc);
           float skj = 1.0f;
           if (FP8) {
             const int j = u.kbeg + i * kM + kl;
             skj = j < sp.T ? p.s_k[(int64_t)u.b * sp.T + j] : 0.0f;
           }
-          float* st = strip + (size_t)slot * QT * CS + pos + kl;
+          float* st = strip + (size_t)slot * QT * CS + (size_t)half * QH * CS + pos + kl;
 #pragma unroll
-          for (int qi = 0; qi < QT; ++qi) {
-            float s = acc[qi].x + acc[qi].y;
+          for (int ql = 0; ql < QH; ++ql) {
+            float s = 0.0f;
+#pragma unroll
+            for (int a = 0; a < NA; ++a) s += acc[ql][a].x + acc[ql][a].y;
             if (FP8) s *= skj;
-            st[(size_t)qi * CS] = s;
+            st[(size_t)ql * CS] = s;
           }
         }
         pos += kM;
@@ -462,7 +493,7 @@ ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
   const int QT = kN / H;
   const size_t q_bytes = (size_t)kN * D * esz;
   const size_t kc_bytes = (size_t)kM * D * esz;
-  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * 4 * kN +
+  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * kEpiWarps * kHalfN +
                        sizeof(ScoreCtlSmem);
   const int cap_min = ((K + 64 + 31) / 32) * 32;
   const int cap_max = ((2 * K + 31) / 32) * 32 > cap_min ? ((2 * K + 31) / 32) * 32 : cap_min;

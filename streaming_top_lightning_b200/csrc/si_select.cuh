@@ -246,6 +246,12 @@ static __device__ __noinline__ bool pool_prune(uint64_t* pool, int* np_io, int K
 // Consume one strip of scores for one query: keys j0 + p, p < nkeys; only
 // keys j < V are visible.  Keys above theta join the pool; a full pool is
 // shrunk to its K best by pool_shrink, which also raises theta.
+// Each lane reads two adjacent scores per step (one 8-byte load) and first
+// compares them with theta's score as floats: a key can only beat theta if
+// its score is at least theta's, so steps where no lane passes that test
+// cost a load, two compares and a vote, and only passing keys are encoded
+// and compared exactly.  Requires st 8-byte aligned and a strip buffer of at
+// least nkeys rounded up to 64 floats.
 SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t* pool, int cap,
                             int K, int* np_p, uint64_t* th_p, uint32_t* hist, int lane) {
   int lim = V - j0;
@@ -253,6 +259,8 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
   if (lim <= 0) return;
   uint64_t theta = *th_p;
   int np = *np_p;
+  // theta 0 takes every key (-inf >= -inf too)
+  float thf = theta ? key_score(theta) : __int_as_float(0xFF800000);
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int p0 = 0; p0 < lim; p0 += 64) {
     // room for this step's up to 64 keys; else raise theta first
@@ -262,12 +270,16 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
         theta = pool_shrink(pool, np, K, hist, lane);
         np = K;
       }
+      thf = key_score(theta);
     }
-    const int pa = p0 + lane, pb = p0 + 32 + lane;
-    const bool va = pa < lim, vb = pb < lim;
-    const uint64_t ka = va ? make_key(st[pa], j0 + pa) : 0ull;
-    const uint64_t kb = vb ? make_key(st[pb], j0 + pb) : 0ull;
-    const bool ta = va && ka > theta, tb = vb && kb > theta;
+    const int pa = p0 + 2 * lane;
+    const float2 v = *reinterpret_cast<const float2*>(st + pa);
+    const bool ca = pa < lim && v.x >= thf;
+    const bool cb = pa + 1 < lim && v.y >= thf;
+    if (!__any_sync(0xFFFFFFFFu, ca || cb)) continue;
+    const uint64_t ka = make_key(v.x, j0 + pa);
+    const uint64_t kb = make_key(v.y, j0 + pa + 1);
+    const bool ta = ca && ka > theta, tb = cb && kb > theta;
     const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta), mb = __ballot_sync(0xFFFFFFFFu, tb);
     const int na = __popc(ma);
     if (ta) pool[np + __popc(ma & lt_mask)] = ka;

@@ -22,27 +22,33 @@ namespace si {
 
 constexpr int kMergeWarps = 4;
 
-// Append the keys of one partial list that beat theta.
+// Append the keys of one partial list that beat theta.  Eight keys per lane
+// (256 per warp) are loaded before any is appended, so their global-memory
+// latencies overlap.
 SI_DEV void pool_take_keys(const uint64_t* keys, int n, uint64_t* pool, int cap, int K, int& np,
                            uint64_t& theta, uint32_t* hist, int lane) {
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r0 = 0; r0 < n; r0 += 64) {
-    if (np + 64 > cap) {
-      __syncwarp();
-      if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
-        theta = pool_shrink(pool, np, K, hist, lane);
-        np = K;
-      }
+  for (int r0 = 0; r0 < n; r0 += 256) {
+    uint64_t k[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = r0 + u * 32 + lane;
+      k[u] = r < n ? __ldg(keys + r) : 0ull;
     }
-    const int ra = r0 + lane, rb = r0 + 32 + lane;
-    const uint64_t ka = ra < n ? keys[ra] : 0ull;
-    const uint64_t kb = rb < n ? keys[rb] : 0ull;
-    const bool ta = ka > theta, tb = kb > theta;  // 0 (padding) never beats theta
-    const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta), mb = __ballot_sync(0xFFFFFFFFu, tb);
-    const int na = __popc(ma);
-    if (ta) pool[np + __popc(ma & lt_mask)] = ka;
-    if (tb) pool[np + na + __popc(mb & lt_mask)] = kb;
-    np += na + __popc(mb);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (np + 32 > cap) {
+        __syncwarp();
+        if (!pool_prune(pool, &np, K, &theta, lane) || np + 32 > cap) {
+          theta = pool_shrink(pool, np, K, hist, lane);
+          np = K;
+        }
+      }
+      const bool tk = k[u] > theta;  // 0 (padding) never beats theta
+      const uint32_t mk = __ballot_sync(0xFFFFFFFFu, tk);
+      if (tk) pool[np + __popc(mk & lt_mask)] = k[u];
+      np += __popc(mk);
+    }
   }
   __syncwarp();
 }

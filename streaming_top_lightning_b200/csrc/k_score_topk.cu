@@ -485,7 +485,7 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
 // CS keys per query, the selection pools (cap keys per query) and the small
 // control block.  Candidates are ranked lexicographically: a pool of at least
 // 1.5K keys first (fewer radix selects), then 3 stages, then strips of 512
-// keys, then the larger pool and more stages.
+// keys, then the larger pool (up to 4K keys) and more stages.
 ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
   ScorePlan best{};
   best.ok = false;
@@ -496,7 +496,7 @@ ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
   const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * kEpiWarps * kHalfN +
                        sizeof(ScoreCtlSmem);
   const int cap_min = ((K + 64 + 31) / 32) * 32;
-  const int cap_max = ((2 * K + 31) / 32) * 32 > cap_min ? ((2 * K + 31) / 32) * 32 : cap_min;
+  const int cap_max = std::max(cap_min, 4 * K);
   const int cs_max = std::min(1024, std::max(128, 4096 / QT));
   long best_score[5] = {-1, -1, -1, -1, -1};
   for (int nst = 2; nst <= 6; ++nst) {

@@ -84,3 +84,16 @@ def test_large_s64k_sampled_rows():
     rows = synth.sample_rows(sh)
     _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
     _gpu.structural(sh, gi, gs, np.arange(0, sh.S, 61))
+
+
+def test_long_s256k_sampled_rows():
+    # S = 262,144 (T = 65,536, top-2048): the sampled rows against the oracle,
+    # and the structural invariants on a stride of rows
+    sh = synth.shape("long_s256k")
+    q = synth.gen_q(sh, 0, threads=16)
+    w = synth.gen_w(sh, 0)
+    kc = synth.gen_kc(sh, 0)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    rows = synth.sample_rows(sh)
+    _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    _gpu.structural(sh, gi, gs, np.arange(0, sh.S, 509))

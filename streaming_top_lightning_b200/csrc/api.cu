@@ -190,7 +190,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
       fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tm_q, tm_kc;
   const int T = pl.T;
-  if ((rc = make_map(&tm_q, q, dt, (uint64_t)B * S * H, D, esz, sw_bytes / esz, 256, sw)))
+  if ((rc = make_map(&tm_q, q, dt, (uint64_t)B * S * H, D, esz, sw_bytes / esz, sp_plan.nq, sw)))
     return rc;
   if ((rc = make_map(&tm_kc, kc, dt, (uint64_t)B * (T > 0 ? T : 1), D, esz, sw_bytes / esz, 128,
                      sw)))
@@ -222,7 +222,8 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     if (grid < 1) grid = 1;
     if (blk == 0 && o.ev_begin && cudaEventRecord(o.ev_begin, stream) != cudaSuccess)
       return SI_ERR_CUDA;
-    if (launch_score_topk(fp8, D, H, tm_q, tm_kc, p, grid, sp_plan.smem, stream) != cudaSuccess)
+    if (launch_score_topk(fp8, D, H, sp_plan.nq, tm_q, tm_kc, p, grid, sp_plan.smem, stream) !=
+        cudaSuccess)
       return SI_ERR_CUDA;
     if (blk + 1 == pl.n_blocks && o.ev_end && cudaEventRecord(o.ev_end, stream) != cudaSuccess)
       return SI_ERR_CUDA;
@@ -243,9 +244,10 @@ int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_o
   if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
   Opts o;
   if ((rc = read_opts(opt, &o))) return rc;
-  const int QT = 256 / H;
-  const Plan pl = make_plan(B, S, S / m, K, QT, o);
-  *bytes = pl.ws_bytes();
+  // the larger need of the two query-tile widths the score plan may choose
+  const Plan full = make_plan(B, S, S / m, K, 256 / H, o);
+  const Plan half = make_plan(B, S, S / m, K, 128 / H, o);
+  *bytes = std::max(full.ws_bytes(), half.ws_bytes());
   (void)fp8;
   return SI_OK;
 }

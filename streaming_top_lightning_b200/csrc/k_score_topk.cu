@@ -35,12 +35,12 @@ namespace si {
 
 constexpr int kThreads = 448;
 constexpr int kRing = 4;        // unit ring depth
-constexpr int kN = 256;         // MMA N: query-tile rows (QT * H)
+constexpr int kN = 256;         // largest MMA N: query-tile rows (QT * H)
 constexpr int kM = 128;         // MMA M: keys per tile
 constexpr int kEpiWarp0 = 2;    // first epilogue warp
 constexpr int kEpiWarps = 8;    // two per TMEM lane quadrant, one per column half
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kHalfN = kN / 2;  // accumulator columns per epilogue warp
+constexpr int kHalfN = kN / 2;  // largest accumulator column count per epilogue warp
 constexpr int kSelWarp0 = kEpiWarp0 + kEpiWarps;  // first selection warp
 static_assert(kThreads == (kSelWarp0 + kSelWarps) * 32, "warp roles");
 
@@ -61,14 +61,14 @@ struct ScoreCtlSmem {
   uint32_t abort;
 };
 
-template <bool FP8, int D>
+template <bool FP8, int D, int NQ>
 struct OperandGeom {
   static constexpr int kEsz = FP8 ? 1 : 2;
   static constexpr int kRowBytes = D * kEsz;                      // bytes of one row
   static constexpr int kSw = kRowBytes >= 128 ? 128 : kRowBytes;  // swizzle span
   static constexpr int kKBlocks = kRowBytes / kSw;                // K-blocks per row
   static constexpr int kKSteps = kRowBytes / 32;                  // MMA instructions per tile
-  static constexpr int kQBytes = kN * kRowBytes;
+  static constexpr int kQBytes = NQ * kRowBytes;
   static constexpr int kKcBytes = kM * kRowBytes;
 };
 
@@ -92,10 +92,11 @@ SI_DEV void tmem_ld_fence(float (&v)[32]) {
 }
 
 // Independent packed accumulators per query of an epilogue warp: enough
-// chains to cover the FMA latency, at most 8 float2 in all.
-template <int H>
+// chains to cover the FMA latency, at most 8 float2 in all.  HALF is the
+// warp's column count (half of the MMA N).
+template <int H, int HALF>
 struct EpiGeom {
-  static constexpr int kQH = kHalfN / H;               // queries per column half
+  static constexpr int kQH = HALF / H;                 // queries per column half
   static constexpr int kNA = kQH >= 8 ? 1 : 8 / kQH;   // chains per query
   static_assert(kQH * kNA <= 16 && (H / 2) % kNA == 0, "accumulator split");
 };
@@ -104,10 +105,10 @@ struct EpiGeom {
 // into the packed accumulators.  Local column c = ch*32 + e is query c / H of
 // the half and head c % H; head pair (c % H)/2 feeds chain ((c % H)/2) % kNA.
 // w4 holds the half's weights as float4 groups (one LDS.128 per 4 columns).
-template <int H>
+template <int H, int HALF>
 SI_DEV void epi_chunk(int ch, const float (&v)[32], const float4* w4,
-                      float2 (&acc)[EpiGeom<H>::kQH][EpiGeom<H>::kNA]) {
-  constexpr int NA = EpiGeom<H>::kNA;
+                      float2 (&acc)[EpiGeom<H, HALF>::kQH][EpiGeom<H, HALF>::kNA]) {
+  constexpr int NA = EpiGeom<H, HALF>::kNA;
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const int col = ch * 32 + e;
@@ -121,12 +122,13 @@ SI_DEV void epi_chunk(int ch, const float (&v)[32], const float4* w4,
   }
 }
 
-template <bool FP8, int D, int H>
+template <bool FP8, int D, int H, int NQ>
 __global__ void __launch_bounds__(kThreads, 1)
     k_score_topk(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                  const ScoreParams p) {
-  using G = OperandGeom<FP8, D>;
-  constexpr int QT = kN / H;
+  using G = OperandGeom<FP8, D, NQ>;
+  constexpr int QT = NQ / H;
+  constexpr int HALF = NQ / 2;  // accumulator columns per epilogue warp
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrow = (b * sp.S + g * QT) * H;
 #pragma unroll
         for (int kb = 0; kb < G::kKBlocks; ++kb)
-          tma_load_2d(q_addr + kb * (kN * G::kSw), &tm_q, qb, kb * (G::kSw / G::kEsz), qrow, pol_q);
+          tma_load_2d(q_addr + kb * (NQ * G::kSw), &tm_q, qb, kb * (G::kSw / G::kEsz), qrow, pol_q);
         q_issued = true;
         ++q_it;
         // key tiles
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = FP8 ? idesc_make(0, 0, kM, kN) : idesc_make(1, 1, kM, kN);
+      constexpr uint32_t idesc = FP8 ? idesc_make(0, 0, kM, NQ) : idesc_make(1, 1, kM, NQ);
       uint32_t ring_it = 0, kstage = 0, acc_it = 0, q_it = 0;
       for (;;) {
         const int r = ring_it % kRing;
@@ -289,14 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t d_tmem = tmem + ab * kN;
+          const uint32_t d_tmem = tmem + ab * NQ;
           const uint32_t a0 = kc_addr + s * G::kKcBytes;
 #pragma unroll
           for (int k = 0; k < G::kKSteps; ++k) {
             constexpr int kPerBlock = G::kSw / 32;
             const int kb = k / kPerBlock, kin = k % kPerBlock;
             const uint64_t ad = sdesc<G::kSw>(a0 + kb * (kM * G::kSw) + kin * 32);
-            const uint64_t bd = sdesc<G::kSw>(q_addr + kb * (kN * G::kSw) + kin * 32);
+            const uint64_t bd = sdesc<G::kSw>(q_addr + kb * (NQ * G::kSw) + kin * 32);
             if (FP8) umma_f8(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
             else umma_bf16(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
           }
@@ -317,8 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kSelWarp0) {
     // ---------------------------------------------------------- epilogue
-    using EG = EpiGeom<H>;
+    using EG = EpiGeom<H, HALF>;
     constexpr int QH = EG::kQH, NA = EG::kNA;
+    static_assert(HALF == 128 || HALF == 64, "epilogue chunk schedule");
     const int ew = warp - kEpiWarp0;  // 0..7
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int half = ew >> 2;         // column half: queries [half*QH, half*QH + QH)
@@ -345,8 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the unit's weights (FP8: folded with the query row scales, which are
       // positive, so relu(s*x) = s*relu(x))
       const int64_t wrow = (int64_t)u.b * sp.S + (int64_t)u.g * QT;
-      for (int i = lane; i < kHalfN; i += 32) {
-        const int col = half * kHalfN + i;  // column of the 256-wide tile
+      for (int i = lane; i < HALF; i += 32) {
+        const int col = half * HALF + i;  // column of the query tile's N columns
         float wv = 0.0f;
         if (u.g * QT + col / H < sp.S) {
           wv = p.w[wrow * H + col];
@@ -374,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t taddr =
-              tmem + ((uint32_t)(quad * 32) << 16) + ab * kN + half * kHalfN;
+              tmem + ((uint32_t)(quad * 32) << 16) + ab * NQ + half * HALF;
           float2 acc[QH][NA];
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql)
@@ -386,19 +389,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           tmem_ld_fence(va);
           tmem_ld_fence(vb);
-          epi_chunk<H>(0, va, w4, acc);
-          tmem_ld32(taddr + 64, va);
-          epi_chunk<H>(1, vb, w4, acc);
-          tmem_ld32(taddr + 96, vb);
-          tmem_ld_wait();
-          tmem_ld_fence(va);
-          tmem_ld_fence(vb);
+          if constexpr (HALF == 128) {
+            epi_chunk<H, HALF>(0, va, w4, acc);
+            tmem_ld32(taddr + 64, va);
+            epi_chunk<H, HALF>(1, vb, w4, acc);
+            tmem_ld32(taddr + 96, vb);
+            tmem_ld_wait();
+            tmem_ld_fence(va);
+            tmem_ld_fence(vb);
+          }
           // every column of this accumulator is in registers: release it
           tc_fence_before();
           mbar_arrive(smem_u32(&cs->acc_empty[ab]));
           ++acc_it;
-          epi_chunk<H>(2, va, w4, acc);
-          epi_chunk<H>(3, vb, w4, acc);
+          epi_chunk<H, HALF>(HALF / 32 - 2, va, w4, acc);
+          epi_chunk<H, HALF>(HALF / 32 - 1, vb, w4, acc);
           float skj = 1.0f;
           if (FP8) {
             const int j = u.kbeg + i * kM + kl;
@@ -446,52 +451,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool FP8, int D, int H>
+template <bool FP8, int D, int H, int NQ>
 static cudaError_t launch_t(const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
                             const ScoreParams& p, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = k_score_topk<FP8, D, H>;
+  auto kern = k_score_topk<FP8, D, H, NQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, stream>>>(tm_q, tm_kc, p);
   return cudaGetLastError();
 }
 
-template <bool FP8, int D>
+template <bool FP8, int D, int NQ>
 static cudaError_t launch_h(int H, const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
                             const ScoreParams& p, int grid, size_t smem, cudaStream_t stream) {
   switch (H) {
-    case 8: return launch_t<FP8, D, 8>(tm_q, tm_kc, p, grid, smem, stream);
-    case 16: return launch_t<FP8, D, 16>(tm_q, tm_kc, p, grid, smem, stream);
-    case 32: return launch_t<FP8, D, 32>(tm_q, tm_kc, p, grid, smem, stream);
-    case 64: return launch_t<FP8, D, 64>(tm_q, tm_kc, p, grid, smem, stream);
+    case 8: return launch_t<FP8, D, 8, NQ>(tm_q, tm_kc, p, grid, smem, stream);
+    case 16: return launch_t<FP8, D, 16, NQ>(tm_q, tm_kc, p, grid, smem, stream);
+    case 32: return launch_t<FP8, D, 32, NQ>(tm_q, tm_kc, p, grid, smem, stream);
+    case 64: return launch_t<FP8, D, 64, NQ>(tm_q, tm_kc, p, grid, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
+template <bool FP8, int D>
+static cudaError_t launch_n(int H, int nq, const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
+                            const ScoreParams& p, int grid, size_t smem, cudaStream_t stream) {
+  if (nq == 256) return launch_h<FP8, D, 256>(H, tm_q, tm_kc, p, grid, smem, stream);
+  if (nq == 128) return launch_h<FP8, D, 128>(H, tm_q, tm_kc, p, grid, smem, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
                               size_t smem, cudaStream_t stream) {
   if (fp8) {
-    if (D == 128) return launch_h<true, 128>(H, tm_q, tm_kc, p, grid, smem, stream);
-    if (D == 64) return launch_h<true, 64>(H, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 128) return launch_n<true, 128>(H, nq, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 64) return launch_n<true, 64>(H, nq, tm_q, tm_kc, p, grid, smem, stream);
   } else {
-    if (D == 128) return launch_h<false, 128>(H, tm_q, tm_kc, p, grid, smem, stream);
-    if (D == 64) return launch_h<false, 64>(H, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 128) return launch_n<false, 128>(H, nq, tm_q, tm_kc, p, grid, smem, stream);
+    if (D == 64) return launch_n<false, 64>(H, nq, tm_q, tm_kc, p, grid, smem, stream);
   }
   return cudaErrorInvalidValue;
 }
 
-// Shared-memory plan: the query tile, NST key-tile stages, two score strips of
-// CS keys per query, the selection pools (cap keys per query) and the small
-// control block.  Candidates are ranked lexicographically: a pool of at least
-// 1.5K keys first (fewer radix selects), then 3 stages, then strips of 512
-// keys, then the larger pool (up to 4K keys) and more stages.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
+// Shared-memory plan for one MMA width NQ: the query tile (NQ rows), NST
+// key-tile stages, two score strips of CS keys per query, the selection pools
+// (cap keys per query) and the small control block.  Candidates are ranked
+// lexicographically: a pool of at least 1.5K keys first (fewer radix
+// selects), then 3 stages, then strips of 512 keys, then the larger pool (up
+// to 4K keys) and more stages.
+static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ) {
   ScorePlan best{};
   best.ok = false;
   const int esz = fp8 ? 1 : 2;
-  const int QT = kN / H;
-  const size_t q_bytes = (size_t)kN * D * esz;
+  const int QT = NQ / H;
+  const size_t q_bytes = (size_t)NQ * D * esz;
   const size_t kc_bytes = (size_t)kM * D * esz;
   const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * kEpiWarps * kHalfN +
                        sizeof(ScoreCtlSmem);
@@ -518,6 +532,7 @@ ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
       if (better) {
         for (int i = 0; i < 5; ++i) best_score[i] = sc[i];
         best.QT = QT;
+        best.nq = NQ;
         best.CS = cs;
         best.nst = nst;
         best.cap = cap;
@@ -527,6 +542,19 @@ ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
     }
   }
   return best;
+}
+
+// The full-width tile (N = 256: 256/H_I queries) is used when its pools can
+// hold 1.5K keys per query; otherwise, for large top-k, the half-width tile
+// (N = 128) halves the queries per tile and so doubles each query's pool,
+// which keeps pruning rare, at the price of reading each key tile from shared
+// memory for half as many columns.
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
+  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN);
+  if (full.ok && full.cap >= (3 * K) / 2) return full;
+  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2);
+  if (half.ok && (!full.ok || half.cap > full.cap)) return half;
+  return full;
 }
 
 }  // namespace si

@@ -25,7 +25,8 @@ struct ScoreParams {
 
 // Shared-memory plan of the fused kernel for one problem shape.
 struct ScorePlan {
-  int QT;        // queries per tile (256 / H)
+  int QT;        // queries per tile (nq / H)
+  int nq;        // MMA N: query-tile rows (QT * H), 256 or 128
   int CS;        // keys per score strip
   int nst;       // pipeline stages
   int cap;       // selection pool entries per query
@@ -35,7 +36,7 @@ struct ScorePlan {
 
 ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem);
 
-cudaError_t launch_score_topk(bool fp8, int D, int H, const CUtensorMap& tm_q,
+cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
                               size_t smem, cudaStream_t stream);
 

@@ -28,6 +28,23 @@ def test_quantize_bit_exact():
     assert torch.all(zc == 0) and torch.all(zs == 1.0)
 
 
+@pytest.mark.parametrize("rows,cols", [(37, 64), (1001, 128), (5, 256), (7, 136), (3, 4096)])
+def test_quantize_shapes_bit_exact(rows, cols):
+    # the lane-group kernels (64, 128, 256 values per row, ragged row counts)
+    # and the warp-per-row kernel (any other length), against the oracle
+    g = np.random.default_rng(rows * 7919 + cols)
+    x = g.standard_normal((rows, cols)).astype(np.float32)
+    x[0] *= 1e-30  # tiny values: codes underflow to zero / subnormals
+    x[-1] = 0.0     # an all-zero row has scale 1
+    if rows > 2:
+        x[1] *= 1e30  # huge values
+    bits = synth.f32_to_bf16_bits(x)
+    codes, scale = stl.quantize_fp8_rows(_gpu.to_dev_bf16(bits))
+    oc, os_ = oracle.quantize_e4m3_rows(bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oc)
+    np.testing.assert_array_equal(scale.cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
 def _fp8_case(sh, seed, rows, opts=None):
     q, w, kc = _gpu.inputs(sh, seed=seed)
     q8, sq = stl.quantize_fp8_rows(_gpu.to_dev_bf16(q))

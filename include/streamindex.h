@@ -30,8 +30,12 @@
  *  - Device-side waits are bounded; a kernel that gives up records a device
  *    error word, read back by si_get_last_device_error().
  *  - Limits: B >= 1; S >= 1 with S % m == 0; H_I in {8, 16, 32, 64};
- *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I*d_I < 2^31 elements per
- *    tensor row index; pointers 16-byte aligned.
+ *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I < 2^31; pointers 16-byte
+ *    aligned.  The selection keeps a candidate pool per query of a query
+ *    tile in shared memory, so with few heads (many queries per tile) the
+ *    largest topk is lower: bf16 H_I=8: 768 (d_I=128), 1152 (d_I=64);
+ *    bf16 H_I=16, d_I=128: 1728; FP8 H_I=8: 1152 (d_I=128), 1344 (d_I=64);
+ *    2048 otherwise.  A larger topk returns SI_ERR_TOPK.
  */
 #ifndef STREAMINDEX_H
 #define STREAMINDEX_H
@@ -47,7 +51,7 @@ extern "C" {
 #define SI_OK 0
 #define SI_ERR_NULL -1           /* a required pointer is NULL */
 #define SI_ERR_DIM -2            /* a dimension is out of range (see limits above) */
-#define SI_ERR_TOPK -3           /* topk < 1 or topk > 2048 */
+#define SI_ERR_TOPK -3           /* topk < 1, > 2048, or above the shape's limit */
 #define SI_ERR_ALIGN -4          /* a pointer is not 16-byte aligned */
 #define SI_ERR_WORKSPACE -5      /* caller workspace too small */
 #define SI_ERR_CUDA -6           /* a CUDA runtime/driver call or launch failed */

@@ -171,7 +171,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
   const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem);
-  if (!sp_plan.ok) return SI_ERR_DIM;
+  if (!sp_plan.ok) return SI_ERR_TOPK;  // the selection pools of this topk do not fit
   const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
   if (!aligned16(ws)) return SI_ERR_ALIGN;

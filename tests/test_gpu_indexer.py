@@ -47,6 +47,30 @@ def test_small_shapes(B, S, m, H, D, k):
     _gpu.structural(sh, gi, gs, rows)
 
 
+@pytest.mark.parametrize("S,H,D,k", [(2048, 64, 128, 1200), (4096, 8, 128, 512), (8704, 32, 64, 2048)])
+def test_half_width_tiles(S, H, D, k):
+    # top-k large enough for the half-width (N = 128) query tile: two (H=64),
+    # four (H=32) or sixteen (H=8) queries per tile; sampled rows including
+    # the last ones, which see more than k keys
+    sh = synth.small(1, S, 4, H, D, k, seed=S + k, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=S + k)
+    gi, gs = _gpu.run_bf16(sh, q, w, kc)
+    rows = np.union1d(np.arange(0, S, 37), np.arange(S - 96, S))
+    _gpu.check_rows(sh, q, w, kc, gi, gs, rows)
+    _gpu.structural(sh, gi, gs, np.arange(S))
+
+
+def test_topk_above_the_shape_limit_is_rejected():
+    # with eight heads a 256-column query tile holds 32 queries; their pools
+    # cannot hold top-1024 candidates each
+    sh = synth.small(1, 512, 4, 8, 128, 1024, seed=1)
+    q, w, kc = _gpu.inputs(sh, seed=1)
+    with pytest.raises(stl.StreamIndexError) as e:
+        _gpu.run_bf16(sh, q, w, kc)
+    assert e.value.status == -3
+
+
+
 @pytest.mark.parametrize("chunk", [128, 256, 1024])
 def test_chunked_equals_unchunked(chunk):
     """Chunking changes only where the selection happens, not the fp32 scores,

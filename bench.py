@@ -209,6 +209,10 @@ def kernel_launches_per_step(sh, args) -> int:
     C = args.key_chunk if args.key_chunk else (sh.T + 127) // 128 * 128
     nch = max(1, (sh.T + C - 1) // C)
     L = (sh.topk + sh.topk // 4 + 64 + 31) // 32 * 32
+    if nch == 1 and args.row_finish == 1:
+        # rows finished in the fused kernel: one launch, no merge
+        n = 1 + (1 if sh.topk > 512 else 0)
+        return n + (2 if args.fp8 else 0)
     per_tile = sh.B * nch * QT * L * 8
     tb = max(1, min(G, (512 << 20) // per_tile))
     n_blocks = (G + tb - 1) // tb
@@ -219,6 +223,8 @@ def kernel_launches_per_step(sh, args) -> int:
 def config_of(sh, args):
     return {"workload": sh.name, "B": sh.B, "S": sh.S, "T": sh.T, "m": sh.m, "H_I": sh.H,
             "d_I": sh.D, "topk": sh.topk, "key_chunk": args.key_chunk,
+            "row_finish": {0: "library choice", 1: "fused kernel", 2: "merge kernel"}[args.row_finish],
+            "key_tile": args.key_tile or "library choice",
             "score_path": "fp8-e4m3" if args.fp8 else "bf16",
             "pairs_per_step": causal_pairs(sh.S, sh.T, sh.m),
             "l2": "inputs larger than L2: q alone is "
@@ -271,7 +277,8 @@ def run_native(args, sh):
     q_d = q_h.to(dev).view(torch.bfloat16)
     w_d = w_h.to(dev)
     kc_d = kc_h.to(dev).view(torch.bfloat16)
-    opts = stl.options(key_chunk=args.key_chunk)
+    opts = stl.options(key_chunk=args.key_chunk, row_finish=args.row_finish,
+                       key_tile=args.key_tile)
     timed = {"opts": None}
 
     def step_opts():
@@ -321,7 +328,8 @@ def run_native(args, sh):
         a.record(stream)
         b.record(stream)
     torch.cuda.synchronize()
-    kopts = [stl.options(key_chunk=args.key_chunk, score_events=e) for e in kev]
+    kopts = [stl.options(key_chunk=args.key_chunk, score_events=e, row_finish=args.row_finish,
+                         key_tile=args.key_tile) for e in kev]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
         barrier()
@@ -445,6 +453,11 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="v4flash_s16k", choices=sorted(synth.SHAPES))
     ap.add_argument("--key-chunk", type=int, default=0)
+    ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
+                    help="1: rows finished in the fused kernel; 2: by the merge kernel; "
+                         "0: the library's choice")
+    ap.add_argument("--key-tile", type=int, default=0, choices=(0, 128, 256, 512),
+                    help="keys per score strip handed to the selection warps (0: library's choice)")
     ap.add_argument("--topk", type=int, default=0)
     ap.add_argument("--fp8", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

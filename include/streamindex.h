@@ -33,8 +33,8 @@
  *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I < 2^31; pointers 16-byte
  *    aligned.  The selection keeps a candidate pool per query of a query
  *    tile in shared memory, so with few heads (many queries per tile) the
- *    largest topk is lower: bf16 H_I=8: 768 (d_I=128), 1152 (d_I=64);
- *    bf16 H_I=16, d_I=128: 1728; FP8 H_I=8: 1152 (d_I=128), 1344 (d_I=64);
+ *    largest topk is lower: bf16 H_I=8: 640 (d_I=128), 1024 (d_I=64);
+ *    bf16 H_I=16, d_I=128: 1600; FP8 H_I=8: 1024 (d_I=128), 1216 (d_I=64);
  *    2048 otherwise.  A larger topk returns SI_ERR_TOPK.
  */
 #ifndef STREAMINDEX_H
@@ -65,7 +65,7 @@ extern "C" {
 typedef struct si_options {
   int key_chunk;        /* keys per chunk of the partition-merge driver, a
                            multiple of 128; 0 = one chunk spans all keys of a
-                           query (no merge pass).  Default 0. */
+                           query.  Default 0. */
   int scratch_mb;       /* bound on partial-list scratch (MiB) used to size the
                            query blocks of the chunked driver.  Default 512. */
   int grid_ctas;        /* persistent CTAs; 0 = one per SM.  Default 0. */
@@ -81,6 +81,17 @@ typedef struct si_options {
                            blocks, the merge launches between them fall
                            inside the interval.  The events stay owned by
                            the caller. */
+  int row_finish;       /* where a query's exact top-k row is finished when
+                           one chunk spans all its keys: 1 = by the fused
+                           kernel's selection warps (no partial lists, no
+                           merge launch), 2 = by the merge kernel from the
+                           fused kernel's pruned candidate lists, 0 = the
+                           library's choice.  With several chunks the merge
+                           kernel always finishes.  Default 0. */
+  int key_tile;         /* keys per score strip handed from the tensor-core
+                           epilogue to the selection warps: 128, 256 or 512
+                           (one to four 128-key MMA tiles); 0 = the library's
+                           choice.  Default 0. */
 } si_options;
 
 /* ---- the indexer step ------------------------------------------------ */
@@ -156,7 +167,8 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
  *   64 MiB device array inside the library (SI_NOALLOC_SCRATCH_BYTES), which
  *   every GPU that loads the library holds until the process exits.  Query
  *   tiles are processed in blocks sized to that array; a problem whose single
- *   query tile needs more than it returns SI_ERR_WORKSPACE.
+ *   query tile needs more returns SI_ERR_WORKSPACE.  That size check comes
+ *   before the pointer checks, so it can be queried with NULL tensors.
  *   The first call on each device looks up the array's device address (once
  *   per device, with that device current); make that first call before any
  *   stream capture.

@@ -88,13 +88,15 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t 
 }
 
 struct Opts {
-  int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags;
+  int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags, row_finish, key_tile;
   cudaEvent_t ev_begin, ev_end;
 };
 
 int read_opts(const si_options* o, Opts* out) {
-  Opts d{0, 512, 0, 2000, 0, nullptr, nullptr};
+  Opts d{0, 512, 0, 2000, 0, 0, 0, nullptr, nullptr};
   if (o) {
+    d.row_finish = o->row_finish;
+    d.key_tile = o->key_tile;
     d.ev_begin = static_cast<cudaEvent_t>(o->score_events[0]);
     d.ev_end = static_cast<cudaEvent_t>(o->score_events[1]);
     d.key_chunk = o->key_chunk;
@@ -103,18 +105,22 @@ int read_opts(const si_options* o, Opts* out) {
     d.timeout_ms = o->timeout_ms > 0 ? o->timeout_ms : 2000;
     d.debug_flags = o->debug_flags;
   }
-  if (d.key_chunk < 0 || (d.key_chunk % 128) != 0 || d.grid_ctas < 0 || d.scratch_mb > (1 << 20))
+  if (d.key_chunk < 0 || (d.key_chunk % 128) != 0 || d.grid_ctas < 0 || d.scratch_mb > (1 << 20) ||
+      d.row_finish < 0 || d.row_finish > 2 ||
+      !(d.key_tile == 0 || d.key_tile == 128 || d.key_tile == 256 || d.key_tile == 512))
     return SI_ERR_OPTIONS;
   *out = d;
   return SI_OK;
 }
 
-// The plan of one problem: tiles, chunks and query blocks.  Every (tile,
-// chunk) unit leaves an L-key partial list per query; the query tiles of one
-// launch block share a scratch of B * tb * nch_max * QT * L keys, sized to the
-// scratch budget, so the scratch does not grow with S.
+// The plan of one problem: tiles, chunks and query blocks.  With several key
+// chunks every (tile, chunk) unit leaves an L-key partial list per query; the
+// query tiles of one launch block share a scratch of B * tb * nch_max * QT * L
+// keys, sized to the scratch budget, so the scratch does not grow with S.
+// With one chunk per tile (final_rows) the selection warps write the output
+// rows themselves: no partial lists, one launch block, no merge.
 struct Plan {
-  int QT, G, T, C, nch_max, L, tb, n_blocks;
+  int QT, G, T, C, nch_max, L, tb, n_blocks, final_rows;
   size_t counters_bytes, partial_bytes;
   size_t ws_bytes() const { return align256(counters_bytes) + partial_bytes; }
 };
@@ -129,16 +135,39 @@ Plan make_plan(int B, int S, int T, int K, int QT, const Opts& o) {
   p.nch_max = T > 0 ? (T + p.C - 1) / p.C : 1;
   if (p.nch_max < 1) p.nch_max = 1;
   p.L = partial_len(K);
-  const size_t per_tile = (size_t)B * p.nch_max * QT * p.L * sizeof(uint64_t);
-  const size_t budget = (size_t)o.scratch_mb << 20;
-  size_t tb = budget / per_tile;
-  if (tb < 1) tb = 1;
-  if (tb > (size_t)p.G) tb = p.G;
-  p.tb = (int)tb;
-  p.partial_bytes = per_tile * p.tb;
-  p.n_blocks = (p.G + p.tb - 1) / p.tb;
+  // rows finished in the fused kernel only on request for now: four
+  // selection warps per SM finish rows far slower than the merge kernel's
+  // many warps (the choice for 0)
+  p.final_rows = (p.nch_max == 1 && o.row_finish == 1) ? 1 : 0;
+  if (p.final_rows) {
+    p.tb = p.G;
+    p.partial_bytes = 0;
+    p.n_blocks = 1;
+  } else {
+    const size_t per_tile = (size_t)B * p.nch_max * QT * p.L * sizeof(uint64_t);
+    const size_t budget = (size_t)o.scratch_mb << 20;
+    size_t tb = budget / per_tile;
+    if (tb < 1) tb = 1;
+    if (tb > (size_t)p.G) tb = p.G;
+    p.tb = (int)tb;
+    p.partial_bytes = per_tile * p.tb;
+    p.n_blocks = (p.G + p.tb - 1) / p.tb;
+  }
   p.counters_bytes = sizeof(int);  // one unit counter shared by every launch
   return p;
+}
+
+// The rows of a query block: from a single candidate list per query (one
+// key chunk) the bucket-sort kernel, else the merge kernel over the chunks.
+cudaError_t finish_launch(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
+                          cudaStream_t stream) {
+  if (sp.nch_max == 1) return launch_finish_rows(partial, sp, stream);
+  return launch_merge(partial, sp, ug, stream);
+}
+
+// True when no row-sort pass is needed after the finishing launches.
+bool rows_come_sorted(const Plan& pl, int K) {
+  return rows_sorted_in_warp(K) || (!pl.final_rows && pl.nch_max == 1);
 }
 
 int check_common(int B, int S, int m, int topk) {
@@ -170,7 +199,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   if ((rc = read_opts(opt, &o))) return rc;
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
-  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem);
+  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile);
   if (!sp_plan.ok) return SI_ERR_TOPK;  // the selection pools of this topk do not fit
   const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
@@ -206,7 +235,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     ScoreParams p{};
     p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
                       sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,
-                      out_idx, out_score, partial};
+                      out_idx, out_score, partial, pl.final_rows};
     p.ug = ug;
     p.w = w;
     p.s_q = s_q;
@@ -215,6 +244,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     p.err = dev->err;
     p.timeout_ns = (uint64_t)o.timeout_ms * 1000000ull;
     p.nst = sp_plan.nst;
+    p.nslot = sp_plan.nslot;
     p.debug_flags = o.debug_flags;
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
@@ -228,10 +258,11 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     if (blk + 1 == pl.n_blocks && o.ev_end && cudaEventRecord(o.ev_end, stream) != cudaSuccess)
       return SI_ERR_CUDA;
     id_base += units + grid;
-    if (launch_merge(partial, p.sel, ug, stream) != cudaSuccess) return SI_ERR_CUDA;
+    if (!pl.final_rows && finish_launch(partial, p.sel, ug, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
   }
-  // rows of more than 512 keys leave the merge unsorted; order them
-  if (!merge_sorts_rows(K) &&
+  // rows of more than 512 keys are written unsorted; order them
+  if (!rows_come_sorted(pl, K) &&
       launch_sort_rows(out_idx, out_score, (int64_t)B * S, K, dev->sms, stream) != cudaSuccess)
     return SI_ERR_CUDA;
   return SI_OK;
@@ -255,7 +286,7 @@ int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_o
 // ------------------------------------------------------------ fixed scratch
 // Device scratch for si_indexer_topk_noalloc: a file-scope array, so the call
 // needs no allocation.  Every GPU that loads the library holds it until exit.
-constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+constexpr size_t kNoAllocScratchBytes = SI_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
@@ -407,7 +438,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base};
     SelParams sp{B,    S,       T,          m,       topk,    QT,     CS,
                  cap,  pl.L,    g_lo,       n_tiles, pl.nch_max, out_idx, out_score,
-                 partial};
+                 partial, pl.final_rows};
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -415,11 +446,11 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     if (launch_topk_scores(scores, sp, ug, counters, dev->err,
                            (uint64_t)o.timeout_ms * 1000000ull, grid, st) != cudaSuccess)
       rc = SI_ERR_CUDA;
-    else if (launch_merge(partial, sp, ug, st) != cudaSuccess)
+    else if (!pl.final_rows && finish_launch(partial, sp, ug, st) != cudaSuccess)
       rc = SI_ERR_CUDA;
     id_base += units + grid;
   }
-  if (rc == SI_OK && !merge_sorts_rows(topk) &&
+  if (rc == SI_OK && !rows_come_sorted(pl, topk) &&
       launch_sort_rows(out_idx, out_score, (int64_t)B * S, topk, dev->sms, st) != cudaSuccess)
     rc = SI_ERR_CUDA;
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;
@@ -439,14 +470,15 @@ int si_get_last_device_error(void* stream) {
 int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B, int S, int H_I,
                             int d_I, int m, int topk, int32_t* out_idx, float* out_score,
                             void* stream) {
-  int rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score);
-  if (rc) return rc;
-  // query blocks sized to the fixed scratch (its last MiB left for the counter)
+  // query blocks sized to the fixed scratch (its last MiB left for the
+  // counter); this size check comes first, so NULL tensors may query it
   si_options opt{};
   opt.scratch_mb = (int)(kNoAllocScratchBytes >> 20) - 1;
   size_t need = 0;
-  if ((rc = workspace_for(false, S, B, H_I, d_I, m, topk, &opt, &need))) return rc;
+  int rc = workspace_for(false, S, B, H_I, d_I, m, topk, &opt, &need);
+  if (rc) return rc;
   if (need > kNoAllocScratchBytes) return SI_ERR_WORKSPACE;  // one query tile does not fit
+  if ((rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score))) return rc;
   void* ws = nullptr;
   if ((rc = noalloc_scratch(&ws))) return rc;
   return run_indexer(false, q, nullptr, w, kc, nullptr, B, S, H_I, d_I, m, topk, out_idx,

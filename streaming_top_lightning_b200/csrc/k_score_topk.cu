@@ -14,7 +14,8 @@
 //
 // Warp roles (448 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer and unit scheduler: takes (tile, chunk) units from
-//               a global counter, loads the query tile once per unit and streams
+//               a global counter one unit ahead (starting the next unit's query
+//               tile towards L2), loads the query tile once per unit and streams
 //               128-key tiles of kc through an NST-stage mbarrier ring;
 //   warp 1      allocates 512 TMEM columns and issues tcgen05.mma (one thread)
 //               into two 256-column accumulators used alternately;
@@ -194,8 +195,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool q_issued = false;
       bool skipped = false;  // debug: one key tile deliberately never loaded
       int skipped_stage = -1;
+      // units are taken one ahead: the next one is known while this one
+      // streams, so its query tile can be on its way to L2.  A CTA stops at
+      // its first failed decode, so the counter still advances by exactly
+      // (units + grid) per launch.
+      int next_id = atomicAdd(p.counter, 1) - p.ug.id_base;
       for (;;) {
-        const int id = atomicAdd(p.counter, 1) - p.ug.id_base;
+        const int id = next_id;
         int b = 0, g = 0, c = 0;
         const bool ok = unit_decode(p.ug, id, b, g, c);
         const int r = ring_it % kRing;
@@ -215,6 +221,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&cs->unit_full[r]));
         ++ring_it;
         if (!ok) break;
+        next_id = atomicAdd(p.counter, 1) - p.ug.id_base;
+        {
+          int b2 = 0, g2 = 0, c2 = 0;
+          if (unit_decode(p.ug, next_id, b2, g2, c2) && (b2 != b || g2 != g)) {
+            const int qrow2 = (b2 * sp.S + g2 * QT) * H;
+#pragma unroll
+            for (int kb = 0; kb < G::kKBlocks; ++kb)
+              tma_prefetch_l2_2d(&tm_q, kb * (G::kSw / G::kEsz), qrow2);
+          }
+        }
         if (u.ntiles == 0) continue;
         // query tile: rows (b*S + g*QT)*H .. +256 of q viewed as [B*S*H, D]
         if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl)) break;
@@ -424,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (pos >= CS || last) {
           if (ew == 0 && lane == 0) {
             const int nk = max(0, min(CS, u.kend - j_strip));
-            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0};
+            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0, 0u};
           }
           mbar_arrive(smem_u32(&cs->strip_full[slot]));
           ++strip_it;
@@ -440,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.meta = cs->meta;
     sm.full_bar = smem_u32(&cs->strip_full[0]);
     sm.empty_bar = smem_u32(&cs->strip_empty[0]);
+    sm.nslot = 2;
     select_loop(sp, sm, ctl, warp - kSelWarp0, lane);
   }
 
@@ -495,12 +512,12 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap&
 }
 
 // Shared-memory plan for one MMA width NQ: the query tile (NQ rows), NST
-// key-tile stages, two score strips of CS keys per query, the selection pools
-// (cap keys per query) and the small control block.  Candidates are ranked
+// key-tile stages, two score strips of CS keys per query (cs_req > 0 fixes
+// CS), the selection pools (cap keys per query) and the small control block.  Candidates are ranked
 // lexicographically: a pool of at least 1.5K keys first (fewer radix
 // selects), then 3 stages, then strips of 512 keys, then the larger pool (up
 // to 4K keys) and more stages.
-static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ) {
+static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ, int cs_req) {
   ScorePlan best{};
   best.ok = false;
   const int esz = fp8 ? 1 : 2;
@@ -515,6 +532,7 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
   long best_score[5] = {-1, -1, -1, -1, -1};
   for (int nst = 2; nst <= 6; ++nst) {
     for (int cs = 128; cs <= cs_max; cs <<= 1) {
+      if (cs_req > 0 && cs != cs_req) continue;
       const size_t used = fixed + nst * kc_bytes + sizeof(float) * 2 * QT * cs;
       if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
       int cap = cap_min;
@@ -535,6 +553,7 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
         best.nq = NQ;
         best.CS = cs;
         best.nst = nst;
+        best.nslot = 2;
         best.cap = cap;
         best.smem = used + sel_state_bytes(QT, cap);
         best.ok = true;
@@ -549,10 +568,10 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
 // (N = 128) halves the queries per tile and so doubles each query's pool,
 // which keeps pruning rare, at the price of reading each key tile from shared
 // memory for half as many columns.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem) {
-  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN);
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req) {
+  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req);
   if (full.ok && full.cap >= (3 * K) / 2) return full;
-  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2);
+  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req);
   if (half.ok && (!full.ok || half.cap > full.cap)) return half;
   return full;
 }

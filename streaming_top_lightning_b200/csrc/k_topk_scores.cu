@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   sm.meta = meta;
   sm.full_bar = full_bar;
   sm.empty_bar = empty_bar;
+  sm.nslot = 2;
 
   if (warp >= kLoadThreads / 32) {
     select_loop(sp, sm, ctl, warp - kLoadThreads / 32, lane);
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
           const float* src = X + ((int64_t)b * sp.S + t) * sp.T + j0;
           for (int q = tid; q < lim; q += kLoadThreads) st[(size_t)qi * CS + q] = __ldg(src + q);
         }
-        if (tid == 0) meta[slot] = StripMeta{1, b, g, c, j0, nk, last};
+        if (tid == 0) meta[slot] = StripMeta{1, b, g, c, j0, nk, last, 0u};
         mbar_arrive(full_bar + 8 * slot);
         ++it;
         if (last) break;

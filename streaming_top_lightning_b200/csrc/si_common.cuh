@@ -153,6 +153,13 @@ SI_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int 
       "l"(map), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
       : "memory");
 }
+// Start moving one tile towards L2 (no shared-memory destination, no
+// completion to wait for).
+SI_DEV void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
 SI_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

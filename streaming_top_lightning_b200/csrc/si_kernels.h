@@ -20,6 +20,7 @@ struct ScoreParams {
   uint32_t* err;       // device error word
   uint64_t timeout_ns; // limit of any single wait
   int nst;             // key-tile pipeline stages
+  int nslot;           // strip ring slots
   int debug_flags;     // bit 0: skip the first key-tile load (timeout test)
 };
 
@@ -29,12 +30,14 @@ struct ScorePlan {
   int nq;        // MMA N: query-tile rows (QT * H), 256 or 128
   int CS;        // keys per score strip
   int nst;       // pipeline stages
+  int nslot;     // strip ring slots
   int cap;       // selection pool entries per query
   size_t smem;   // dynamic shared memory bytes
   bool ok;
 };
 
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem);
+// cs_req: keys per score strip (128, 256 or 512), 0 = the planner's choice.
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req);
 
 cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,
@@ -50,6 +53,10 @@ cudaError_t launch_merge(const uint64_t* partial, const SelParams& sp, const Uni
 
 // True when the merge kernel already writes sorted rows (small K).
 bool merge_sorts_rows(int K);
+
+// Exact sorted rows from a single candidate list per query (one key chunk);
+// every row comes out sorted, whatever K.
+cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, cudaStream_t stream);
 
 // Sorts each of the rows [rows, K] of (idx, score) in place into the output
 // order (score descending, index ascending, padding last).

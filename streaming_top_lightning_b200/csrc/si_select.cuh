@@ -32,6 +32,7 @@ struct StripMeta {
   int j0;      // first key of the strip
   int nkeys;   // keys in the strip (<= CS)
   int last;    // 1 if this is the unit's last strip
+  uint32_t seq;  // the producer's running unit number
 };
 
 struct SelParams {
@@ -43,6 +44,8 @@ struct SelParams {
   int32_t* out_idx;    // [B,S,K]
   float* out_score;    // [B,S,K]
   uint64_t* partial;   // [B, n_tiles, nch_max, QT, L] candidate keys, 0-padded
+  int final_rows;      // 1: every tile is one unit, whose pools are final: the selection
+                       // warps write the exact top-K rows themselves (no partial lists)
 };
 
 // A unit leaves at most this many candidates per query (a superset of its K
@@ -55,10 +58,11 @@ struct SelSmem {
   uint64_t* theta;     // [QT] current threshold
   int* npool;          // [QT] keys in each pool
   uint32_t* hist;      // [kSelWarps][8][32] digit counters of each selection warp
-  float* strip;        // [2][QT][CS]
-  StripMeta* meta;     // [2]
-  uint32_t full_bar;   // 2 mbarriers, 8 bytes apart
-  uint32_t empty_bar;  // 2 mbarriers, 8 bytes apart
+  float* strip;        // [nslot][QT][CS] scores
+  StripMeta* meta;     // [nslot]
+  uint32_t full_bar;   // nslot mbarriers, 8 bytes apart
+  uint32_t empty_bar;  // nslot mbarriers, 8 bytes apart
+  int nslot;           // strip slots in the ring (2..8)
 };
 
 SI_DEV int visible_keys(int t, int T, int m) {
@@ -320,15 +324,125 @@ SI_DEV void warp_emit(const SelParams& p, const StripMeta& md, int qi, const uin
   __syncwarp();
 }
 
+// ------------------------------------------------------------------ row sort
+// Bitonic sort of 32*R keys held by one warp, blocked layout: lane l holds
+// elements l*R .. l*R+R-1 in v[0..R).  Distances below R pair registers of one
+// lane; larger ones pair lanes through xor-shuffles.  The lower index of each
+// pair keeps the max where (index & size) == 0, so the result is descending.
+template <int R, int S>
+SI_DEV void bsort_reg(uint64_t (&v)[R], int lane, int size) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if ((r & S) == 0) {
+      const bool dir = ((lane * R + r) & size) == 0;
+      const uint64_t a = v[r], b = v[r | S];
+      const bool gt = a > b;
+      const uint64_t mx = gt ? a : b, mn = gt ? b : a;
+      v[r] = dir ? mx : mn;
+      v[r | S] = dir ? mn : mx;
+    }
+  }
+}
+
+template <int R>
+SI_DEV void warp_sort_blocked(uint64_t (&v)[R], int lane) {
+#pragma unroll 1
+  for (int size = 2; size <= 32 * R; size <<= 1) {
+#pragma unroll 1
+    for (int s = size >> 1; s > 0; s >>= 1) {
+      if (s >= R) {
+        const int lm = s / R;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const bool dir = ((lane * R + r) & size) == 0;
+          const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, v[r], lm);
+          const bool gt = v[r] > y;
+          v[r] = ((lower == dir) == gt) ? v[r] : y;
+        }
+      } else if (s == 8) {
+        if constexpr (R > 8) bsort_reg<R, 8>(v, lane, size);
+      } else if (s == 4) {
+        if constexpr (R > 4) bsort_reg<R, 4>(v, lane, size);
+      } else if (s == 2) {
+        if constexpr (R > 2) bsort_reg<R, 2>(v, lane, size);
+      } else {
+        if constexpr (R > 1) bsort_reg<R, 1>(v, lane, size);
+      }
+    }
+  }
+}
+
+// Sort the n (<= 32*R) keys in pool[0, n) and write the first K of them as an
+// output row (index, score), padded with -1 / -inf.  The pool is unsorted, so
+// reading it lane-interleaved (conflict-free) and treating that as the
+// blocked layout loses nothing.
+template <int R>
+SI_DEV void sort_and_write(const uint64_t* pool, int n, int K, int32_t* oi, float* os, int lane) {
+  uint64_t v[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int i = 32 * r + lane;
+    v[r] = i < n ? pool[i] : 0ull;
+  }
+  warp_sort_blocked<R>(v, lane);
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int e = lane * R + r;
+    if (e < K) {
+      const uint64_t k = v[r];
+      oi[e] = k ? key_index(k) : -1;
+      os[e] = k ? key_score(k) : __int_as_float(0xFF800000);
+    }
+  }
+}
+
+// Final output row from a pool that holds a superset of the row's K best keys
+// (np of them): the exact K best (prune, then the radix select), sorted in
+// registers for K <= 512; larger rows are written unsorted and ordered by the
+// row-sort kernel afterwards.
+static __device__ __noinline__ void finish_row(uint64_t* pool, int np, int K, uint32_t* hist,
+                                               int32_t* oi, float* os, int lane) {
+  __syncwarp();
+  if (np > K) {
+    uint64_t th;
+    while (np > K + K / 4 + 64 && pool_prune(pool, &np, K, &th, lane)) {
+    }
+    if (np > K) pool_shrink(pool, np, K, hist, lane);
+    np = K;
+  }
+  __syncwarp();
+  switch (pow2ceil(K < 32 ? 32 : K)) {
+    case 32: sort_and_write<1>(pool, np, K, oi, os, lane); break;
+    case 64: sort_and_write<2>(pool, np, K, oi, os, lane); break;
+    case 128: sort_and_write<4>(pool, np, K, oi, os, lane); break;
+    case 256: sort_and_write<8>(pool, np, K, oi, os, lane); break;
+    case 512: sort_and_write<16>(pool, np, K, oi, os, lane); break;
+    default:
+      for (int r = lane; r < K; r += 32) {
+        const bool real = r < np;
+        const uint64_t k = real ? pool[r] : 0ull;
+        oi[r] = real ? key_index(k) : -1;
+        os[r] = real ? key_score(k) : __int_as_float(0xFF800000);
+      }
+  }
+  __syncwarp();
+}
+
+// True when finish_row() leaves the row sorted (else the row-sort kernel runs).
+__host__ __device__ constexpr bool rows_sorted_in_warp(int K) { return K <= 512; }
+
 // The selection warps' loop: take filled strips in order until a strip says
 // there is no more work (or the CTA aborts).  Query qi belongs to selection
 // warp qi % kSelWarps for the whole kernel, so its pool, threshold and count
-// are only ever touched by that warp.
+// are only ever touched by that warp.  At a unit's last strip the warp either
+// writes the exact output row itself (final_rows: the unit covers all of the
+// query's keys) or leaves a pruned partial list for the merge kernel.
 SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, int sw, int lane) {
   uint32_t* hist = sm.hist + sw * 256;
   for (uint32_t it = 0;; ++it) {
-    const int slot = it & 1;
-    const uint32_t ph = (it >> 1) & 1u;
+    const int slot = (int)(it % (uint32_t)sm.nslot);
+    const uint32_t ph = (it / (uint32_t)sm.nslot) & 1u;
     if (!mbar_wait_warp(sm.full_bar + 8 * slot, ph, ctl)) return;
     const StripMeta md = sm.meta[slot];  // ordered after the acquiring wait
     if (!md.valid) return;
@@ -340,8 +454,13 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
       pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), pool,
                       p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane);
       if (md.last) {
-        const int n = pool_trim(pool, sm.npool[qi], p.K, p.L, hist, lane);
-        warp_emit(p, md, qi, pool, n, lane);
+        if (p.final_rows) {
+          const int64_t o = ((int64_t)md.b * p.S + t) * p.K;
+          finish_row(pool, sm.npool[qi], p.K, hist, p.out_idx + o, p.out_score + o, lane);
+        } else {
+          const int n = pool_trim(pool, sm.npool[qi], p.K, p.L, hist, lane);
+          warp_emit(p, md, qi, pool, n, lane);
+        }
         if (lane == 0) {
           sm.npool[qi] = 0;
           sm.theta[qi] = 0ull;

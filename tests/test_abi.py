@@ -67,11 +67,32 @@ def test_workspace_size_and_validation(lib):
     assert _ws(lib, 1, 16384, 64, 128, 4, 512, _lib.SiOptions(100, 0, 0, 0, 0))[0] == -8
 
 
-def test_null_and_alignment_rejected_before_cuda(lib):
+def test_noalloc_size_check_comes_first(lib):
+    # one query tile over B=1024 batches with top-2048 needs about 86 MB of
+    # partial-list scratch (1024 batches x 4 queries x 2624 candidates x 8
+    # bytes), more than the fixed 64 MiB array: refused before any pointer is
+    # looked at (the tensors here are NULL, so a problem that fits is then
+    # refused for its NULL pointers, and nothing can reach a launch)
     P = ctypes.c_void_p
-    ok = P(0x1000)
-    assert lib.si_indexer_topk(None, ok, ok, 1, 64, 8, 64, 4, 8, ok, ok, None) == -1
-    assert lib.si_indexer_topk(P(0x1001), ok, ok, 1, 64, 8, 64, 4, 8, ok, ok, None) == -4
-    assert lib.si_indexer_topk(ok, ok, ok, 1, 64, 8, 64, 4, 9999, ok, ok, None) == -3
-    assert lib.si_topk_scores(None, 1, 4, 4, 1, 2, ok, ok, None, None) == -1
-    assert lib.si_quantize_fp8_rows(ok, 4, 12, ok, ok, None) == -2
+    assert lib.si_indexer_topk_noalloc(None, None, None, 1024, 8192, 64, 128, 4, 2048,
+                                       None, None, None) == -5
+    assert lib.si_indexer_topk_noalloc(None, None, None, 1, 8192, 64, 128, 4, 2048,
+                                       None, None, None) == -1
+    assert lib.si_indexer_topk_noalloc(P(0x1000), P(0x1000), P(0x1000), 1, 8191, 64, 128, 4,
+                                       512, P(0x1000), P(0x1000), None) == -2
+
+
+def test_row_finish_option(lib):
+    # rows finished in the fused kernel need no partial lists: the workspace
+    # is the unit counter alone, whatever the problem size
+    for B, S, H, D, k in [(1, 262144, 64, 128, 2048), (64, 65536, 8, 64, 64)]:
+        o = _lib.SiOptions(0, 0, 0, 0, 0)
+        o.row_finish = 1
+        rc, n = _ws(lib, B, S, H, D, 4, k, o)
+        assert rc == 0 and 0 < n <= 256
+        o.row_finish = 2
+        rc, n2 = _ws(lib, B, S, H, D, 4, k, o)
+        assert rc == 0 and n2 > 256
+    o = _lib.SiOptions(0, 0, 0, 0, 0)
+    o.row_finish = 3
+    assert _ws(lib, 1, 16384, 64, 128, 4, 512, o)[0] == -8

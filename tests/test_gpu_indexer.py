@@ -83,6 +83,22 @@ def test_chunked_equals_unchunked(chunk):
     assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
 
 
+@pytest.mark.parametrize("B,S,m,H,D,k", [(1, 2048, 4, 8, 64, 64), (2, 1024, 4, 64, 128, 100),
+                                         (1, 4096, 4, 64, 128, 512), (1, 2048, 4, 64, 128, 1200)])
+def test_rows_finished_in_fused_kernel_equal_merge(B, S, m, H, D, k):
+    """Finishing the rows in the fused kernel's selection warps or in the
+    merge kernel selects from the same fp32 scores under the same total
+    order, so the two return exactly the same rows (sorted in registers for
+    k <= 512, by the row-sort kernel above)."""
+    sh = synth.small(B, S, m, H, D, k, seed=S + k, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=S + k)
+    gi0, gs0 = _gpu.run_bf16(sh, q, w, kc, opts=stl.options(row_finish=2))
+    gi1, gs1 = _gpu.run_bf16(sh, q, w, kc, opts=stl.options(row_finish=1))
+    assert torch.equal(gi0, gi1)
+    assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
+    _gpu.structural(sh, gi1, gs1, np.arange(B * S))
+
+
 def test_repeatable():
     sh = synth.small(1, 4096, 4, 64, 128, 512, seed=4, kc_kind="ar1")
     q, w, kc = _gpu.inputs(sh, seed=4)

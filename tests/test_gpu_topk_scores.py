@@ -41,6 +41,22 @@ def test_bit_exact(kind, B, S, T, m, k, chunk):
     np.testing.assert_array_equal(gs.view(np.uint32), os_.view(np.uint32))
 
 
+@pytest.mark.parametrize("kind", ["normal", "ties", "inf"])
+@pytest.mark.parametrize("B,S,T,m,k,chunk", [c for c in CASES if c[5] == 0])
+def test_bit_exact_rows_finished_by_selection_warps(kind, B, S, T, m, k, chunk):
+    """With one key chunk the selection warps can finish the rows themselves
+    (exact select, in-register sort for k <= 512, row sort above): still
+    bit-exact against the oracle."""
+    X = synth.gen_scores(B, S, T, seed=B * 7 + S, kind=kind)
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), m, k, opts=stl.options(row_finish=1))
+    torch.cuda.synchronize()
+    assert stl.device_error() == 0
+    oi, os_ = oracle.topk_scores(X, m, k)
+    np.testing.assert_array_equal(gi.reshape(-1, k).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, k).cpu().numpy().view(np.uint32),
+                                  os_.view(np.uint32))
+
+
 def test_increasing_rows_worst_case():
     """Scores rising along j: every key beats the running k-th, so every strip
     overflows the candidate buffer."""

@@ -343,7 +343,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;         // column half: queries [half*QH, half*QH + QH)
     const int kl = quad * 32 + lane;  // key within the tile
     float* wq = w_s + ew * kHalfN;    // this warp's private copy of its half's weights
-    const float4* w4 = reinterpret_cast<const float4*>(wq);
     uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
     for (;;) {
       const int r = ring_it % kRing;
@@ -361,17 +360,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         break;
       }
-      // the unit's weights (FP8: folded with the query row scales, which are
-      // positive, so relu(s*x) = s*relu(x))
+      // the unit's weights.  bf16: read in place from global memory (the
+      // warp's 128 columns are contiguous in w); every lane reads the same
+      // 16 bytes, which costs the L1 one wavefront where a shared-memory
+      // broadcast of 16 bytes costs four, and these reads would otherwise
+      // fill the shared-memory pipe.  FP8 (weights folded with the query row
+      // scales, which are positive, so relu(s*x) = s*relu(x)) and the last,
+      // partial tile of the last batch (whose rows past S lie outside w) take
+      // a zero-padded copy in shared memory.
       const int64_t wrow = (int64_t)u.b * sp.S + (int64_t)u.g * QT;
-      for (int i = lane; i < HALF; i += 32) {
-        const int col = half * HALF + i;  // column of the query tile's N columns
-        float wv = 0.0f;
-        if (u.g * QT + col / H < sp.S) {
-          wv = p.w[wrow * H + col];
-          if (FP8) wv *= p.s_q[wrow * H + col];
+      const bool w_direct = !FP8 && !(u.b == sp.B - 1 && (u.g + 1) * QT > sp.S);
+      const float4* w4 = reinterpret_cast<const float4*>(p.w + wrow * H + half * HALF);
+      if (!w_direct) {
+        for (int i = lane; i < HALF; i += 32) {
+          const int col = half * HALF + i;  // column of the query tile's N columns
+          float wv = 0.0f;
+          if (u.g * QT + col / H < sp.S) {
+            wv = p.w[wrow * H + col];
+            if (FP8) wv *= p.s_q[wrow * H + col];
+          }
+          wq[i] = wv;
         }
-        wq[i] = wv;
+        w4 = reinterpret_cast<const float4*>(wq);
       }
       __syncwarp();
       int pos = 0, j_strip = u.kbeg;

@@ -222,20 +222,42 @@ static __device__ __noinline__ bool pool_prune(uint64_t* pool, int* np_io, int K
   if (r < 0) r = 0;
   for (; r < 32; r += 2) {
     const uint64_t pivot = __shfl_sync(0xFFFFFFFFu, v, r);
+    // both passes take four 32-key groups per iteration, so their loads and
+    // ballots overlap
     int c = 0;
-    for (int i = lane; i < np; i += 32) c += pool[i] >= pivot ? 1 : 0;
+    for (int i0 = 0; i0 < np; i0 += 128) {
+      uint64_t k[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 32 * u + lane;
+        k[u] = i < np ? pool[i] : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c += (i0 + 32 * u + lane < np && k[u] >= pivot) ? 1 : 0;
+    }
     c = __reduce_add_sync(0xFFFFFFFFu, c);
     if (c >= K) {
       if (c >= np) return false;  // nothing to drop
       int w = 0;
       const uint32_t lt_mask = (1u << lane) - 1u;
-      for (int i0 = 0; i0 < np; i0 += 32) {
-        const int i = i0 + lane;
-        const uint64_t k = i < np ? pool[i] : 0ull;
-        const bool take = i < np && k >= pivot;
-        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, take);
-        if (take) pool[w + __popc(tm & lt_mask)] = k;  // forward, in place
-        w += __popc(tm);
+      for (int i0 = 0; i0 < np; i0 += 128) {
+        uint64_t k[4];
+        uint32_t m[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 32 * u + lane;
+          k[u] = i < np ? pool[i] : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          m[u] = __ballot_sync(0xFFFFFFFFu, i0 + 32 * u + lane < np && k[u] >= pivot);
+        // forward, in place: the block's keys are all read before any is
+        // written, and a write position never passes its read position
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (m[u] & (1u << lane)) pool[w + __popc(m[u] & lt_mask)] = k[u];
+          w += __popc(m[u]);
+        }
       }
       __syncwarp();
       *np_io = w;
@@ -248,14 +270,16 @@ static __device__ __noinline__ bool pool_prune(uint64_t* pool, int* np_io, int K
 
 // ------------------------------------------------------------------ strips
 // Consume one strip of scores for one query: keys j0 + p, p < nkeys; only
-// keys j < V are visible.  Keys above theta join the pool; a full pool is
-// shrunk to its K best by pool_shrink, which also raises theta.
-// Each lane reads two adjacent scores per step (one 8-byte load) and first
-// compares them with theta's score as floats: a key can only beat theta if
-// its score is at least theta's, so steps where no lane passes that test
-// cost a load, two compares and a vote, and only passing keys are encoded
-// and compared exactly.  Requires st 8-byte aligned and a strip buffer of at
-// least nkeys rounded up to 64 floats.
+// keys j < V are visible.  Keys whose score is at least theta's join the pool
+// (only those can beat theta; the few extra keys of equal score are
+// harmless); a full pool is pruned, which raises theta.
+// The strip is taken in chunks of eight 64-key steps, lane l reading keys
+// p0 + l and p0 + 32 + l of each step.  A chunk's loads, compares and ballots
+// are all issued before any key is stored, and the steps' pool offsets are
+// uniform prefix sums of the ballot counts, so the chunk's latencies overlap
+// instead of chaining step after step.  When the pool cannot take the next
+// step, the steps that fit are stored, the pool is pruned and the rest of the
+// chunk is compared again with the new threshold.
 SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t* pool, int cap,
                             int K, int* np_p, uint64_t* th_p, uint32_t* hist, int lane) {
   int lim = V - j0;
@@ -266,29 +290,60 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
   // theta 0 takes every key (-inf >= -inf too)
   float thf = theta ? key_score(theta) : __int_as_float(0xFF800000);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int p0 = 0; p0 < lim; p0 += 64) {
-    // room for this step's up to 64 keys; else raise theta first
-    if (np + 64 > cap) {
-      __syncwarp();
-      if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
-        theta = pool_shrink(pool, np, K, hist, lane);
-        np = K;
-      }
-      thf = key_score(theta);
+  constexpr int kSteps = 8;
+  for (int c0 = 0; c0 < lim; c0 += 64 * kSteps) {
+    const float ninf = __int_as_float(0xFF800000);
+    float xa[kSteps], xb[kSteps];
+#pragma unroll
+    for (int u = 0; u < kSteps; ++u) {
+      const int pa = c0 + 64 * u + lane;
+      xa[u] = pa < lim ? st[pa] : ninf;
+      xb[u] = pa + 32 < lim ? st[pa + 32] : ninf;
     }
-    const int pa = p0 + 2 * lane;
-    const float2 v = *reinterpret_cast<const float2*>(st + pa);
-    const bool ca = pa < lim && v.x >= thf;
-    const bool cb = pa + 1 < lim && v.y >= thf;
-    if (!__any_sync(0xFFFFFFFFu, ca || cb)) continue;
-    const uint64_t ka = make_key(v.x, j0 + pa);
-    const uint64_t kb = make_key(v.y, j0 + pa + 1);
-    const bool ta = ca && ka > theta, tb = cb && kb > theta;
-    const uint32_t ma = __ballot_sync(0xFFFFFFFFu, ta), mb = __ballot_sync(0xFFFFFFFFu, tb);
-    const int na = __popc(ma);
-    if (ta) pool[np + __popc(ma & lt_mask)] = ka;
-    if (tb) pool[np + na + __popc(mb & lt_mask)] = kb;
-    np += na + __popc(mb);
+    const int nsteps = min(kSteps, (lim - c0 + 63) >> 6);
+    int s0 = 0;
+    while (s0 < nsteps) {
+      uint32_t ma[kSteps], mb[kSteps];
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        const int pa = c0 + 64 * u + lane;
+        ma[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && pa < lim && xa[u] >= thf);
+        mb[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && pa + 32 < lim && xb[u] >= thf);
+      }
+      // the steps [s0, s1) that fit the pool
+      int s1 = s0, add = 0;
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        const int c = __popc(ma[u]) + __popc(mb[u]);
+        if (u >= s0 && u == s1 && u < nsteps && np + add + c <= cap) {
+          add += c;
+          s1 = u + 1;
+        }
+      }
+      int base = np;
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        if (u >= s0 && u < s1) {
+          const int pa = c0 + 64 * u + lane;
+          const int na = __popc(ma[u]);
+          if (ma[u] & (1u << lane)) pool[base + __popc(ma[u] & lt_mask)] = make_key(xa[u], j0 + pa);
+          if (mb[u] & (1u << lane))
+            pool[base + na + __popc(mb[u] & lt_mask)] = make_key(xb[u], j0 + pa + 32);
+          base += na + __popc(mb[u]);
+        }
+      }
+      np += add;
+      s0 = s1;
+      if (s0 < nsteps) {
+        // the pool cannot take step s0: raise theta, then compare the rest again
+        __syncwarp();
+        if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
+          theta = pool_shrink(pool, np, K, hist, lane);
+          np = K;
+        }
+        thf = key_score(theta);
+      }
+    }
   }
   __syncwarp();
   if (lane == 0) {

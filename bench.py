@@ -225,6 +225,7 @@ def config_of(sh, args):
             "d_I": sh.D, "topk": sh.topk, "key_chunk": args.key_chunk,
             "row_finish": {0: "library choice", 1: "fused kernel", 2: "merge kernel"}[args.row_finish],
             "key_tile": args.key_tile or "library choice",
+            "strip_slots": args.strip_slots or "library choice",
             "score_path": "fp8-e4m3" if args.fp8 else "bf16",
             "pairs_per_step": causal_pairs(sh.S, sh.T, sh.m),
             "l2": "inputs larger than L2: q alone is "
@@ -278,7 +279,7 @@ def run_native(args, sh):
     w_d = w_h.to(dev)
     kc_d = kc_h.to(dev).view(torch.bfloat16)
     opts = stl.options(key_chunk=args.key_chunk, row_finish=args.row_finish,
-                       key_tile=args.key_tile)
+                       key_tile=args.key_tile, strip_slots=args.strip_slots)
     timed = {"opts": None}
 
     def step_opts():
@@ -329,7 +330,7 @@ def run_native(args, sh):
         b.record(stream)
     torch.cuda.synchronize()
     kopts = [stl.options(key_chunk=args.key_chunk, score_events=e, row_finish=args.row_finish,
-                         key_tile=args.key_tile) for e in kev]
+                         key_tile=args.key_tile, strip_slots=args.strip_slots) for e in kev]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
         barrier()
@@ -456,7 +457,9 @@ def main():
     ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
                     help="1: rows finished in the fused kernel; 2: by the merge kernel; "
                          "0: the library's choice")
-    ap.add_argument("--key-tile", type=int, default=0, choices=(0, 128, 256, 512),
+    ap.add_argument("--strip-slots", type=int, default=0, choices=(0, 2, 3, 4),
+                    help="score strips in flight between epilogue and selection (0: library's choice)")
+    ap.add_argument("--key-tile", type=int, default=0, choices=(0, 128, 256, 512, 1024),
                     help="keys per score strip handed to the selection warps (0: library's choice)")
     ap.add_argument("--topk", type=int, default=0)
     ap.add_argument("--fp8", action="store_true")

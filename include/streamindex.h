@@ -33,8 +33,8 @@
  *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I < 2^31; pointers 16-byte
  *    aligned.  The selection keeps a candidate pool per query of a query
  *    tile in shared memory, so with few heads (many queries per tile) the
- *    largest topk is lower: bf16 H_I=8: 640 (d_I=128), 1024 (d_I=64);
- *    bf16 H_I=16, d_I=128: 1600; FP8 H_I=8: 1024 (d_I=128), 1216 (d_I=64);
+ *    largest topk is lower: bf16 H_I=8: 768 (d_I=128), 1152 (d_I=64);
+ *    bf16 H_I=16, d_I=128: 1728; FP8 H_I=8: 1152 (d_I=128), 1344 (d_I=64);
  *    2048 otherwise.  A larger topk returns SI_ERR_TOPK.
  */
 #ifndef STREAMINDEX_H
@@ -89,8 +89,11 @@ typedef struct si_options {
                            library's choice.  With several chunks the merge
                            kernel always finishes.  Default 0. */
   int key_tile;         /* keys per score strip handed from the tensor-core
-                           epilogue to the selection warps: 128, 256 or 512
-                           (one to four 128-key MMA tiles); 0 = the library's
+                           epilogue to the selection warps: 128, 256, 512 or
+                           1024 (one to eight 128-key MMA tiles); 0 = the
+                           library's choice.  Default 0. */
+  int strip_slots;      /* score strips in flight between the epilogue and
+                           the selection warps: 2 to 4; 0 = the library's
                            choice.  Default 0. */
 } si_options;
 

@@ -52,16 +52,18 @@ def _need(t, dtype, ndim, name):
 
 def options(key_chunk: int = 0, scratch_mb: int = 0, grid_ctas: int = 0, timeout_ms: int = 0,
             debug_flags: int = 0, score_events=None, row_finish: int = 0,
-            key_tile: int = 0) -> SiOptions:
+            key_tile: int = 0, strip_slots: int = 0) -> SiOptions:
     """Tuning knobs of include/streamindex.h.  ``score_events`` is an optional
     pair of ``torch.cuda.Event(enable_timing=True)`` that the call records around
     its score-kernel launches (on the call's stream).  ``row_finish``: 1 = rows
     finished in the fused kernel, 2 = by the merge kernel, 0 = the library's
     choice.  ``key_tile``: keys per score strip (128, 256, 512; 0 = the
+    library's choice); ``strip_slots``: score strips in flight (2..4; 0 = the
     library's choice)."""
     o = SiOptions(key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags)
     o.row_finish = row_finish
     o.key_tile = key_tile
+    o.strip_slots = strip_slots
     if score_events is not None:
         a, b = score_events
         o.score_events[0] = a.cuda_event

@@ -30,7 +30,8 @@ class SiOptions(ctypes.Structure):
     _fields_ = [("key_chunk", ctypes.c_int), ("scratch_mb", ctypes.c_int),
                 ("grid_ctas", ctypes.c_int), ("timeout_ms", ctypes.c_int),
                 ("debug_flags", ctypes.c_int), ("score_events", ctypes.c_void_p * 2),
-                ("row_finish", ctypes.c_int), ("key_tile", ctypes.c_int)]
+                ("row_finish", ctypes.c_int), ("key_tile", ctypes.c_int),
+                ("strip_slots", ctypes.c_int)]
 
 
 class StreamIndexError(RuntimeError):

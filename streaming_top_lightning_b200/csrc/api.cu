@@ -88,15 +88,17 @@ int make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t 
 }
 
 struct Opts {
-  int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags, row_finish, key_tile;
+  int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags, row_finish, key_tile,
+      strip_slots;
   cudaEvent_t ev_begin, ev_end;
 };
 
 int read_opts(const si_options* o, Opts* out) {
-  Opts d{0, 512, 0, 2000, 0, 0, 0, nullptr, nullptr};
+  Opts d{0, 512, 0, 2000, 0, 0, 0, 0, nullptr, nullptr};
   if (o) {
     d.row_finish = o->row_finish;
     d.key_tile = o->key_tile;
+    d.strip_slots = o->strip_slots;
     d.ev_begin = static_cast<cudaEvent_t>(o->score_events[0]);
     d.ev_end = static_cast<cudaEvent_t>(o->score_events[1]);
     d.key_chunk = o->key_chunk;
@@ -107,7 +109,9 @@ int read_opts(const si_options* o, Opts* out) {
   }
   if (d.key_chunk < 0 || (d.key_chunk % 128) != 0 || d.grid_ctas < 0 || d.scratch_mb > (1 << 20) ||
       d.row_finish < 0 || d.row_finish > 2 ||
-      !(d.key_tile == 0 || d.key_tile == 128 || d.key_tile == 256 || d.key_tile == 512))
+      !(d.key_tile == 0 || d.key_tile == 128 || d.key_tile == 256 || d.key_tile == 512 ||
+        d.key_tile == 1024) ||
+      d.strip_slots < 0 || d.strip_slots == 1 || d.strip_slots > 4)
     return SI_ERR_OPTIONS;
   *out = d;
   return SI_OK;
@@ -199,7 +203,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   if ((rc = read_opts(opt, &o))) return rc;
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
-  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile);
+  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile, o.strip_slots);
   if (!sp_plan.ok) return SI_ERR_TOPK;  // the selection pools of this topk do not fit
   const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;

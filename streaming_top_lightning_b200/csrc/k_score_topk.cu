@@ -43,6 +43,7 @@ constexpr int kEpiWarps = 8;    // two per TMEM lane quadrant, one per column ha
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kHalfN = kN / 2;  // largest accumulator column count per epilogue warp
 constexpr int kSelWarp0 = kEpiWarp0 + kEpiWarps;  // first selection warp
+constexpr int kMaxSlots = 4;    // score-strip ring slots at most
 static_assert(kThreads == (kSelWarp0 + kSelWarps) * 32, "warp roles");
 
 struct UnitInfo {
@@ -54,10 +55,10 @@ struct ScoreCtlSmem {
   uint64_t acc_full[2], acc_empty[2];
   uint64_t q_full, q_empty;
   uint64_t unit_full[kRing], unit_empty[kRing];
-  uint64_t strip_full[2], strip_empty[2];
+  uint64_t strip_full[kMaxSlots], strip_empty[kMaxSlots];
   uint64_t drain;
   UnitInfo ring[kRing];
-  StripMeta meta[2];
+  StripMeta meta[kMaxSlots];
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -135,13 +136,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const SelParams& sp = p.sel;
-  const int CS = sp.CS, NST = p.nst;
+  const int CS = sp.CS, NST = p.nst, NSL = p.nslot;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   uint8_t* q_s = smem;
   uint8_t* kc_s = q_s + G::kQBytes;
   float* strip = reinterpret_cast<float*>(kc_s + (size_t)NST * G::kKcBytes);
-  uint8_t* sel_base = reinterpret_cast<uint8_t*>(strip + 2 * QT * CS);
+  uint8_t* sel_base = reinterpret_cast<uint8_t*>(strip + (size_t)NSL * QT * CS);
   SelSmem sm;
   sel_state_carve(sel_base, QT, sp.cap, sm);
   // [kEpiWarps][kHalfN]: each epilogue warp's private copy of its half of the weights
@@ -157,6 +158,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&cs->acc_full[i]), 1);
       mbar_init(smem_u32(&cs->acc_empty[i]), kEpiThreads);
+    }
+    for (int i = 0; i < NSL; ++i) {
       mbar_init(smem_u32(&cs->strip_full[i]), kEpiThreads);
       mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);
     }
@@ -353,8 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ring_it;
       if (!u.valid) {
         // no more work: pass the end marker to the selection warps
-        const int slot = strip_it & 1;
-        if (mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it >> 1) & 1u) ^ 1u, ctl)) {
+        const int slot = (int)(strip_it % (uint32_t)NSL);
+        if (mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u, ctl)) {
           if (ew == 0 && lane == 0) cs->meta[slot].valid = 0;
           mbar_arrive(smem_u32(&cs->strip_full[slot]));
         }
@@ -387,9 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pos = 0, j_strip = u.kbeg;
       bool stop = false;
       for (int i = 0; i < u.ntiles || (i == 0 && u.ntiles == 0); ++i) {
-        const int slot = strip_it & 1;
+        const int slot = (int)(strip_it % (uint32_t)NSL);
         if (pos == 0) {
-          if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it >> 1) & 1u) ^ 1u,
+          if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u,
                               ctl)) {
             stop = true;
             break;
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.meta = cs->meta;
     sm.full_bar = smem_u32(&cs->strip_full[0]);
     sm.empty_bar = smem_u32(&cs->strip_empty[0]);
-    sm.nslot = 2;
+    sm.nslot = NSL;
     select_loop(sp, sm, ctl, warp - kSelWarp0, lane);
   }
 
@@ -522,12 +525,15 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap&
 }
 
 // Shared-memory plan for one MMA width NQ: the query tile (NQ rows), NST
-// key-tile stages, two score strips of CS keys per query (cs_req > 0 fixes
-// CS), the selection pools (cap keys per query) and the small control block.  Candidates are ranked
-// lexicographically: a pool of at least 1.5K keys first (fewer radix
-// selects), then 3 stages, then strips of 512 keys, then the larger pool (up
-// to 4K keys) and more stages.
-static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ, int cs_req) {
+// key-tile stages, a ring of NSL score strips of CS keys per query (cs_req and
+// nsl_req > 0 fix them), the selection pools (cap keys per query) and the small
+// control block.  Candidates are ranked lexicographically: a pool of at least
+// 1.5K keys first, then enough stages (below), then strips of 512 keys, then
+// the larger pool up to 4K keys (a prune's cost per accepted key falls as
+// cap / (cap - 1.2K)), then more strip slots, then more stages.  Measured on
+// the V4-Flash-shaped step, pool room beats a third stage and extra slots.
+static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ, int cs_req,
+                              int nsl_req) {
   ScorePlan best{};
   best.ok = false;
   const int esz = fp8 ? 1 : 2;
@@ -539,34 +545,41 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
   const int cap_min = ((K + 64 + 31) / 32) * 32;
   const int cap_max = std::max(cap_min, 4 * K);
   const int cs_max = std::min(1024, std::max(128, 4096 / QT));
-  long best_score[5] = {-1, -1, -1, -1, -1};
+  // key-tile stages wanted: a full-width tile's MMA (1024 cycles at the
+  // dense rate) hides a tile load from L2 with two stages; a half-width
+  // tile's takes half as long and needs three
+  const int min_nst = NQ == kN ? 2 : 3;
+  long best_score[6] = {-1, -1, -1, -1, -1, -1};
   for (int nst = 2; nst <= 6; ++nst) {
     for (int cs = 128; cs <= cs_max; cs <<= 1) {
       if (cs_req > 0 && cs != cs_req) continue;
-      const size_t used = fixed + nst * kc_bytes + sizeof(float) * 2 * QT * cs;
-      if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
-      int cap = cap_min;
-      while (cap + 32 <= cap_max && used + sel_state_bytes(QT, cap + 32) <= (size_t)max_smem)
-        cap += 32;
-      const long sc[5] = {std::min(cap, (3 * K) / 2), std::min(nst, 3), std::min(cs, 512), cap,
-                          nst};
-      bool better = false;
-      for (int i = 0; i < 5; ++i) {
-        if (sc[i] != best_score[i]) {
-          better = sc[i] > best_score[i];
-          break;
+      for (int nsl = 2; nsl <= kMaxSlots; ++nsl) {
+        if (nsl_req > 0 && nsl != nsl_req) continue;
+        const size_t used = fixed + nst * kc_bytes + sizeof(float) * (size_t)nsl * QT * cs;
+        if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
+        int cap = cap_min;
+        while (cap + 32 <= cap_max && used + sel_state_bytes(QT, cap + 32) <= (size_t)max_smem)
+          cap += 32;
+        const long sc[6] = {std::min(cap, (3 * K) / 2), std::min(nst, min_nst), std::min(cs, 512),
+                            std::min(cap, 4 * K), nsl, nst};
+        bool better = false;
+        for (int i = 0; i < 6; ++i) {
+          if (sc[i] != best_score[i]) {
+            better = sc[i] > best_score[i];
+            break;
+          }
         }
-      }
-      if (better) {
-        for (int i = 0; i < 5; ++i) best_score[i] = sc[i];
-        best.QT = QT;
-        best.nq = NQ;
-        best.CS = cs;
-        best.nst = nst;
-        best.nslot = 2;
-        best.cap = cap;
-        best.smem = used + sel_state_bytes(QT, cap);
-        best.ok = true;
+        if (better) {
+          for (int i = 0; i < 6; ++i) best_score[i] = sc[i];
+          best.QT = QT;
+          best.nq = NQ;
+          best.CS = cs;
+          best.nst = nst;
+          best.nslot = nsl;
+          best.cap = cap;
+          best.smem = used + sel_state_bytes(QT, cap);
+          best.ok = true;
+        }
       }
     }
   }
@@ -578,10 +591,10 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
 // (N = 128) halves the queries per tile and so doubles each query's pool,
 // which keeps pruning rare, at the price of reading each key tile from shared
 // memory for half as many columns.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req) {
-  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req);
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req) {
+  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
   if (full.ok && full.cap >= (3 * K) / 2) return full;
-  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req);
+  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
   if (half.ok && (!full.ok || half.cap > full.cap)) return half;
   return full;
 }

@@ -36,8 +36,9 @@ struct ScorePlan {
   bool ok;
 };
 
-// cs_req: keys per score strip (128, 256 or 512), 0 = the planner's choice.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req);
+// cs_req: keys per score strip (128 .. 1024), nsl_req: strip ring slots
+// (2 .. 4); 0 = the planner's choice.
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req);
 
 cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,

@@ -199,25 +199,27 @@ def run_reference(args, sh):
 
 
 def kernel_launches_per_step(sh, args) -> int:
-    """Our kernel launches in one step: a score and a merge launch per query
-    block, the row sort when topk > 512, and the two quantiser launches of the
-    FP8 path.  The query-block count follows the library's scratch plan (512 MiB
-    of partial lists by default; 256/H_I queries per tile; partial lists of
+    """Our kernel launches in one step, following the library's plan: per query
+    block a score launch and a finishing launch (the bucket-sort finish with
+    one key chunk, the merge with several), the row sort when topk > 512 and
+    the merge finished the rows, and the two quantiser launches of the FP8
+    path.  With rows finished in the fused kernel: one score launch (and the
+    row sort above 512).  Query blocks follow the scratch plan (512 MiB of
+    partial lists by default; 256/H_I queries per tile; partial lists of
     ceil((K + K/4 + 64)/32)*32 keys per query and key chunk)."""
     QT = 256 // sh.H
     G = (sh.S + QT - 1) // QT
     C = args.key_chunk if args.key_chunk else (sh.T + 127) // 128 * 128
     nch = max(1, (sh.T + C - 1) // C)
     L = (sh.topk + sh.topk // 4 + 64 + 31) // 32 * 32
+    fp8 = 2 if args.fp8 else 0
     if nch == 1 and args.row_finish == 1:
-        # rows finished in the fused kernel: one launch, no merge
-        n = 1 + (1 if sh.topk > 512 else 0)
-        return n + (2 if args.fp8 else 0)
+        return 1 + (1 if sh.topk > 512 else 0) + fp8
     per_tile = sh.B * nch * QT * L * 8
     tb = max(1, min(G, (512 << 20) // per_tile))
     n_blocks = (G + tb - 1) // tb
-    n = 2 * n_blocks + (1 if sh.topk > 512 else 0)
-    return n + (2 if args.fp8 else 0)
+    sort = 1 if (nch > 1 and sh.topk > 512) else 0
+    return 2 * n_blocks + sort + fp8
 
 
 def config_of(sh, args):

@@ -12,9 +12,10 @@
 // select finds the exact K-th largest pool key, which becomes theta, and the
 // pool is compacted to the K keys at or above it.  A unit (a tile of QT
 // queries x one key chunk) ends by pruning its pool to at most L candidates,
-// written to scratch as the unit's partial list; the merge kernel
-// (k_merge.cu) takes the exact top K over a query's partial lists and the
-// row sort (k_sort_rows.cu) orders the result.
+// written to scratch as the unit's partial list.  With one key chunk the
+// bucket-sort kernel (k_finish.cu) turns each list into the sorted row; with
+// several, the merge kernel (k_merge.cu) takes the exact top K over a query's
+// lists and the row sort (k_sort_rows.cu) orders rows longer than 512.
 // Every pass reads the pool with consecutive lanes on consecutive keys, so no
 // access has bank conflicts.
 #pragma once

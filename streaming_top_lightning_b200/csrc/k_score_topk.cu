@@ -198,18 +198,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool q_issued = false;
       bool skipped = false;  // debug: one key tile deliberately never loaded
       int skipped_stage = -1;
-      // units are taken one ahead: the next one is known while this one
-      // streams, so its query tile can be on its way to L2.  A CTA stops at
-      // its first failed decode, so the counter still advances by exactly
-      // (units + grid) per launch.
-      int next_id = atomicAdd(p.counter, 1) - p.ug.id_base;
-      for (;;) {
-        const int id = next_id;
+      // Units are taken and published one ahead: the next unit's descriptor is
+      // in the ring before this unit's first key tile is loaded, so the MMA
+      // and epilogue warps never wait for it, and its query tile is on its way
+      // to L2 while this one streams.  A CTA stops at its first failed decode
+      // (which it publishes as the end marker), so the counter still advances
+      // by exactly (units + grid) per launch.  The ring has room: its
+      // consumers release an entry when they start that unit, and they are at
+      // most one unit behind the one being loaded.
+      // publish(): 1 = a unit, 0 = the end marker, -1 = abort
+      auto publish = [&](int id, UnitInfo& u) -> int {
         int b = 0, g = 0, c = 0;
         const bool ok = unit_decode(p.ug, id, b, g, c);
         const int r = ring_it % kRing;
-        if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl)) break;
-        UnitInfo u{0, 0, 0, 0, 0, 0, 0};
+        if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl)) return -1;
+        u = UnitInfo{0, 0, 0, 0, 0, 0, 0};
         if (ok) {
           const int vmax = tile_vmax(p.ug, g);
           u.valid = 1;
@@ -223,52 +226,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         cs->ring[r] = u;
         mbar_arrive(smem_u32(&cs->unit_full[r]));
         ++ring_it;
-        if (!ok) break;
-        next_id = atomicAdd(p.counter, 1) - p.ug.id_base;
-        {
-          int b2 = 0, g2 = 0, c2 = 0;
-          if (unit_decode(p.ug, next_id, b2, g2, c2) && (b2 != b || g2 != g)) {
-            const int qrow2 = (b2 * sp.S + g2 * QT) * H;
+        return ok ? 1 : 0;
+      };
+      UnitInfo u;
+      int st = publish(atomicAdd(p.counter, 1) - p.ug.id_base, u);
+      while (st > 0) {
+        UnitInfo nxt;
+        const int st2 = publish(atomicAdd(p.counter, 1) - p.ug.id_base, nxt);
+        if (st2 < 0) break;
+        if (st2 > 0 && nxt.ntiles > 0 && (nxt.b != u.b || nxt.g != u.g)) {
+          const int qrow2 = (nxt.b * sp.S + nxt.g * QT) * H;
 #pragma unroll
-            for (int kb = 0; kb < G::kKBlocks; ++kb)
-              tma_prefetch_l2_2d(&tm_q, kb * (G::kSw / G::kEsz), qrow2);
-          }
+          for (int kb = 0; kb < G::kKBlocks; ++kb)
+            tma_prefetch_l2_2d(&tm_q, kb * (G::kSw / G::kEsz), qrow2);
         }
-        if (u.ntiles == 0) continue;
-        // query tile: rows (b*S + g*QT)*H .. +256 of q viewed as [B*S*H, D]
-        if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl)) break;
-        const uint32_t qb = smem_u32(&cs->q_full);
-        mbar_arrive_expect_tx(qb, G::kQBytes);
-        const int qrow = (b * sp.S + g * QT) * H;
+        if (u.ntiles > 0) {
+          // query tile: rows (b*S + g*QT)*H .. +NQ of q viewed as [B*S*H, D]
+          if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl)) break;
+          const uint32_t qb = smem_u32(&cs->q_full);
+          mbar_arrive_expect_tx(qb, G::kQBytes);
+          const int qrow = (u.b * sp.S + u.g * QT) * H;
 #pragma unroll
-        for (int kb = 0; kb < G::kKBlocks; ++kb)
-          tma_load_2d(q_addr + kb * (NQ * G::kSw), &tm_q, qb, kb * (G::kSw / G::kEsz), qrow, pol_q);
-        q_issued = true;
-        ++q_it;
-        // key tiles
-        bool stop = false;
-        for (int i = 0; i < u.ntiles; ++i) {
-          const int s = kstage % NST;
-          if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl)) {
-            stop = true;
-            break;
-          }
-          const uint32_t fb = smem_u32(&cs->full[s]);
-          mbar_arrive_expect_tx(fb, G::kKcBytes);
-          if ((p.debug_flags & 1) && !skipped) {
-            skipped = true;  // the consumer's wait on this stage must expire
-            skipped_stage = s;
-          } else {
-            const int krow = b * sp.T + u.kbeg + i * kM;
-            const uint32_t dst = kc_addr + s * G::kKcBytes;
+          for (int kb = 0; kb < G::kKBlocks; ++kb)
+            tma_load_2d(q_addr + kb * (NQ * G::kSw), &tm_q, qb, kb * (G::kSw / G::kEsz), qrow,
+                        pol_q);
+          q_issued = true;
+          ++q_it;
+          // key tiles
+          bool stop = false;
+          for (int i = 0; i < u.ntiles; ++i) {
+            const int s = kstage % NST;
+            if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl)) {
+              stop = true;
+              break;
+            }
+            const uint32_t fb = smem_u32(&cs->full[s]);
+            mbar_arrive_expect_tx(fb, G::kKcBytes);
+            if ((p.debug_flags & 1) && !skipped) {
+              skipped = true;  // the consumer's wait on this stage must expire
+              skipped_stage = s;
+            } else {
+              const int krow = u.b * sp.T + u.kbeg + i * kM;
+              const uint32_t dst = kc_addr + s * G::kKcBytes;
 #pragma unroll
-            for (int kb = 0; kb < G::kKBlocks; ++kb)
-              tma_load_2d(dst + kb * (kM * G::kSw), &tm_kc, fb, kb * (G::kSw / G::kEsz), krow,
-                          pol_k);
+              for (int kb = 0; kb < G::kKBlocks; ++kb)
+                tma_load_2d(dst + kb * (kM * G::kSw), &tm_kc, fb, kb * (G::kSw / G::kEsz), krow,
+                            pol_k);
+            }
+            ++kstage;
           }
-          ++kstage;
+          if (stop) break;
         }
-        if (stop) break;
+        u = nxt;
+        st = st2;
       }
       // drain: wait (bounded, regardless of abort) for every copy this thread
       // issued to land before the CTA may exit

@@ -96,3 +96,15 @@ def test_row_finish_option(lib):
     o = _lib.SiOptions(0, 0, 0, 0, 0)
     o.row_finish = 3
     assert _ws(lib, 1, 16384, 64, 128, 4, 512, o)[0] == -8
+
+
+def test_strip_options_validated(lib):
+    for kt, ss, ok in [(0, 0, True), (128, 2, True), (1024, 4, True), (100, 0, False),
+                       (2048, 0, False), (0, 1, False), (0, 5, False), (256, -1, False)]:
+        o = _lib.SiOptions(0, 0, 0, 0, 0)
+        o.key_tile = kt
+        o.strip_slots = ss
+        rc, _ = _ws(lib, 1, 16384, 64, 128, 4, 512, o)
+        assert (rc == 0) == ok, (kt, ss, rc)
+        if not ok:
+            assert rc == -8

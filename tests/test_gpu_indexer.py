@@ -99,6 +99,21 @@ def test_rows_finished_in_fused_kernel_equal_merge(B, S, m, H, D, k):
     _gpu.structural(sh, gi1, gs1, np.arange(B * S))
 
 
+@pytest.mark.parametrize("key_tile,strip_slots", [(128, 2), (256, 3), (512, 4), (1024, 2), (128, 4)])
+def test_strip_options_do_not_change_rows(key_tile, strip_slots):
+    """The strip length and the number of strips in flight change only how the
+    scores travel from the epilogue to the selection warps (and so the pool
+    room the planner leaves), never which keys are selected: the rows are
+    bit-identical to the default plan's."""
+    sh = synth.small(1, 6144, 4, 64, 128, 300, seed=11, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=11)
+    gi0, gs0 = _gpu.run_bf16(sh, q, w, kc)
+    gi1, gs1 = _gpu.run_bf16(sh, q, w, kc,
+                             opts=stl.options(key_tile=key_tile, strip_slots=strip_slots))
+    assert torch.equal(gi0, gi1)
+    assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
+
+
 def test_repeatable():
     sh = synth.small(1, 4096, 4, 64, 128, 512, seed=4, kc_kind="ar1")
     q, w, kc = _gpu.inputs(sh, seed=4)

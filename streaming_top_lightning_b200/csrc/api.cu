@@ -235,7 +235,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   for (int blk = 0; blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base};
+    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, 1};
     ScoreParams p{};
     p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
                       sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,
@@ -328,6 +328,7 @@ int host_tile_chunks(const UnitGrid& u, int g) {
 }
 
 int host_count_units(const UnitGrid& u) {
+  if (u.tile_units) return u.B * u.n_tiles;
   int64_t n = 0;
   for (int g = u.g_lo; g < u.g_lo + u.n_tiles; ++g) n += host_tile_chunks(u, g);
   n *= u.B;
@@ -439,7 +440,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   for (int blk = 0; rc == SI_OK && blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base};
+    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base, 0};
     SelParams sp{B,    S,       T,          m,       topk,    QT,     CS,
                  cap,  pl.L,    g_lo,       n_tiles, pl.nch_max, out_idx, out_score,
                  partial, pl.final_rows};

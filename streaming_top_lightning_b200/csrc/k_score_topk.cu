@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           u.g = g;
           u.c = c;
           u.kbeg = c * p.ug.C;
-          u.kend = min(u.kbeg + p.ug.C, vmax);
+          u.kend = p.ug.tile_units ? vmax : min(u.kbeg + p.ug.C, vmax);
           u.ntiles = u.kend > u.kbeg ? (u.kend - u.kbeg + kM - 1) / kM : 0;
         }
         cs->ring[r] = u;
@@ -398,6 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       int pos = 0, j_strip = u.kbeg;
+      const int sp_chunk = p.ug.C;  // keys per chunk (a multiple of 128)
+      int chunk_next = u.kbeg + sp_chunk;  // end of the current key chunk
+      int chunk_idx = u.kbeg / sp_chunk;
       bool stop = false;
       for (int i = 0; i < u.ntiles || (i == 0 && u.ntiles == 0); ++i) {
         const int slot = (int)(strip_it % (uint32_t)NSL);
@@ -459,16 +462,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         pos += kM;
+        // a strip ends when full, at the end of a key chunk (the selection
+        // then leaves that chunk's partial list) or at the unit's last tile
+        const int jt_end = u.kbeg + (i + 1) * kM;
         const bool last = (i + 1 >= u.ntiles);
-        if (pos >= CS || last) {
+        const bool chunk_end = last || jt_end == chunk_next;
+        if (pos >= CS || chunk_end) {
           if (ew == 0 && lane == 0) {
-            const int nk = max(0, min(CS, u.kend - j_strip));
-            cs->meta[slot] = StripMeta{1, u.b, u.g, u.c, j_strip, nk, last ? 1 : 0, 0u};
+            const int nk = max(0, min(CS, min(chunk_next, u.kend) - j_strip));
+            cs->meta[slot] =
+                StripMeta{1, u.b, u.g, chunk_idx, j_strip, nk, chunk_end ? 1 : 0, 0u};
           }
           mbar_arrive(smem_u32(&cs->strip_full[slot]));
           ++strip_it;
           pos = 0;
-          j_strip += CS;
+          j_strip = jt_end;
+          if (chunk_end) {
+            chunk_next += sp_chunk;
+            ++chunk_idx;
+          }
         }
       }
       if (stop) break;

@@ -549,9 +549,14 @@ SI_DEV void sel_state_carve(uint8_t* p, int QT, int cap, SelSmem& sm) {
 // chunk c of tile g holds keys [c*C, min((c+1)*C, Vmax(g))), where Vmax(g) is
 // the visible count of the tile's last query.  Units are numbered chunk-major;
 // inside a chunk, tiles run from the largest (most keys) down, batch fastest.
+// With tile_units, a unit is a whole tile (all its chunks, in order), tiles
+// again from the largest down.
 struct UnitGrid {
   int B, S, T, m, QT, C, g_lo, n_tiles;
-  int id_base;  // value of the shared unit counter when this launch starts
+  int id_base;     // value of the shared unit counter when this launch starts
+  int tile_units;  // 1: a unit is a whole query tile, its key chunks handled in
+                   // order inside it (the tile is loaded once); 0: one unit
+                   // per (tile, chunk)
 };
 
 SI_DEV int tile_vmax(const UnitGrid& u, int g) {
@@ -571,6 +576,13 @@ SI_DEV int tile_chunks(const UnitGrid& u, int g) {
 SI_DEV bool unit_decode(const UnitGrid& u, int id, int& b, int& g, int& c) {
   if (id < 0) return false;
   const int g_hi = u.g_lo + u.n_tiles;  // exclusive
+  if (u.tile_units) {
+    if (id >= u.B * u.n_tiles) return false;
+    g = g_hi - 1 - id / u.B;
+    b = id % u.B;
+    c = 0;
+    return true;
+  }
   for (int cc = 0;; ++cc) {
     // tiles with more than cc chunks form a suffix [g_first, g_hi)
     int lo = u.g_lo, hi = g_hi;

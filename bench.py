@@ -235,6 +235,36 @@ def config_of(sh, args):
             "parallelism": f"replicas x{args.gpus} (independent problems)"}
 
 
+# --------------------------------------------------------------------------- ranks
+
+
+class Ranks:
+    """The multi-rank plumbing of a weak-scaling run: one process per GPU (or
+    per CPU process under gloo in the tests), each rank solving its own
+    problem.  The only collectives are the timing barrier and the maximum
+    over ranks of a measured time; the whole-job value divides the pairs all
+    ranks processed by that maximum."""
+
+    def __init__(self, dist, world: int, rank: int, device):
+        self.dist, self.world, self.rank, self.device = dist, world, rank, device
+
+    def barrier(self) -> None:
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def job_value(self, pairs_per_rank: int, ms_per_step: float) -> float:
+        return self.world * pairs_per_rank / (ms_per_step / 1e3)
+
+
 # --------------------------------------------------------------------------- native
 
 
@@ -255,16 +285,8 @@ def run_native(args, sh):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(dist, world, rank, dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
 
     seed = rank
     P = causal_pairs(sh.S, sh.T, sh.m)
@@ -357,8 +379,8 @@ def run_native(args, sh):
     # end to end through the public API: host -> device inputs, the call,
     # device -> host result, every step
     if args.no_e2e:
-        return finish(args, sh, world, rank, P, K, total_ms, launch_ms, None, None, None, None,
-                      peak_alloc, free0, free1, clk, dist)
+        return finish(args, sh, ranks, P, K, total_ms, launch_ms, None, None, None, None,
+                      peak_alloc, free0, free1, clk)
     idx_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32).pin_memory()
     score_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32).pin_memory()
     qe = torch.empty_like(q_h, device=dev)
@@ -396,15 +418,16 @@ def run_native(args, sh):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     assert stl.device_error() == 0
-    return finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h,
-                  peak_alloc, free0, free1, clk, dist)
+    return finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h,
+                  peak_alloc, free0, free1, clk)
 
 
-def finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, peak_alloc,
-           free0, free1, clk, dist):
+def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, peak_alloc,
+           free0, free1, clk):
+    world, rank, dist = ranks.world, ranks.rank, ranks.dist
     flops_per_pair = 2 * sh.H * sh.D
     ms_per_step = total_ms / K
-    value = world * P * sh.B / (ms_per_step / 1e3)
+    value = ranks.job_value(P * sh.B, ms_per_step)
     peaks, peak_src = measured_peaks()
     flops_launch = flops_per_pair * P * sh.B
     achieved = flops_launch / (launch_ms / 1e3) / 1e12
@@ -430,7 +453,7 @@ def finish(args, sh, world, rank, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2
                      "algorithmic_flops_per_launch": flops_launch,
                      "avg_launch_ms": launch_ms},
         "e2e": None if e2e_ms is None else {
-            "value": world * P * sh.B * Ke / (e2e_ms / 1e3), "unit": UNIT,
+            "value": ranks.job_value(P * sh.B, e2e_ms / Ke), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": K * launches_per_step,
         "clocks": clk.summary(),

@@ -139,9 +139,9 @@ Plan make_plan(int B, int S, int T, int K, int QT, const Opts& o) {
   p.nch_max = T > 0 ? (T + p.C - 1) / p.C : 1;
   if (p.nch_max < 1) p.nch_max = 1;
   p.L = partial_len(K);
-  // rows finished in the fused kernel only on request for now: four
-  // selection warps per SM finish rows far slower than the merge kernel's
-  // many warps (the choice for 0)
+  // rows finished in the fused kernel only on request: its four selection
+  // warps per SM finish rows far slower than the bucket-sort kernel, which
+  // spreads that work over the whole GPU (the choice for 0)
   p.final_rows = (p.nch_max == 1 && o.row_finish == 1) ? 1 : 0;
   if (p.final_rows) {
     p.tb = p.G;

@@ -78,7 +78,7 @@ typedef struct si_options {
                            score-kernel launch and [1] just after its last
                            one, so cudaEventElapsedTime gives the fused score
                            kernel's own device time.  With several query
-                           blocks, the merge launches between them fall
+                           blocks, the finishing launches between them fall
                            inside the interval.  The events stay owned by
                            the caller. */
   int row_finish;       /* where a query's exact top-k row is finished when

@@ -76,3 +76,36 @@ def test_reference_arm_idle_on_other_ranks(monkeypatch, capsys):
 
     assert bench.run_reference(A, synth.shape("tiny")) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_launch_count_follows_the_plan():
+    # one key chunk: a score and a bucket-sort finishing launch per query
+    # block, no row sort whatever k; several chunks: score + merge per block
+    # and the row sort above k = 512; FP8 adds the two quantiser launches;
+    # rows finished in the fused kernel: one launch (and the sort above 512)
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+
+    class A:
+        key_chunk = 0
+        row_finish = 0
+        fp8 = False
+
+    assert bench.kernel_launches_per_step(synth.shape("v4flash_s16k"), A) == 2
+    assert bench.kernel_launches_per_step(synth.shape("tiny"), A) == 2
+    # top-2048 lists at S = 65,536 need three query blocks of the 512 MiB budget
+    assert bench.kernel_launches_per_step(synth.shape("large_s64k"), A) == 6
+    A.fp8 = True
+    assert bench.kernel_launches_per_step(synth.shape("v4flash_s16k"), A) == 4
+    A.fp8 = False
+    # eight chunks of 1024 keys at S = 32,768: 8 x 4 x 704 x 8 B of lists per
+    # query tile gives three query blocks for top-512; top-1024's longer lists
+    # give six, and the merge leaves rows of more than 512 keys to the row sort
+    A.key_chunk = 1024
+    assert bench.kernel_launches_per_step(synth.shape("sweep_s32k", topk=512), A) == 6
+    assert bench.kernel_launches_per_step(synth.shape("sweep_s32k", topk=1024), A) == 13
+    A.key_chunk = 0
+    A.row_finish = 1
+    assert bench.kernel_launches_per_step(synth.shape("v4flash_s16k"), A) == 1
+    assert bench.kernel_launches_per_step(synth.shape("large_s64k"), A) == 2

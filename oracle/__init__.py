@@ -38,40 +38,66 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def declare(lib):
+    """Declare the argument types of every oracle symbol on a loaded CDLL
+    (the built oracle, or a test's modified copy of it)."""
+    P = ctypes.c_void_p
+    I, L = ctypes.c_int, ctypes.c_int64
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = I
+    lib.oracle_visible.argtypes = [I, I, I]
+    lib.oracle_visible.restype = I
+    lib.oracle_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
+    lib.oracle_indexer_topk.restype = I
+    lib.oracle_indexer_topk_rows.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
+    lib.oracle_indexer_topk_rows.restype = I
+    lib.oracle_indexer_topk_rows_absmax.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P, P]
+    lib.oracle_indexer_topk_rows_absmax.restype = I
+    lib.oracle_score_keys_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, I, P]
+    lib.oracle_score_keys_rows.restype = None
+    lib.oracle_row_absmax_rows.argtypes = [P, P, P, I, I, I, I, P, I, P]
+    lib.oracle_row_absmax_rows.restype = None
+    lib.oracle_topk_scores.argtypes = [P, I, I, I, I, I, P, I, P, P]
+    lib.oracle_topk_scores.restype = I
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_decode.restype = ctypes.c_double
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_quantize_e4m3_rows.argtypes = [P, L, I, P, P]
+    lib.oracle_quantize_e4m3_rows.restype = None
+    lib.oracle_indexer_topk_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, P, P]
+    lib.oracle_indexer_topk_fp8_rows.restype = I
+    lib.oracle_score_keys_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, I, P]
+    lib.oracle_score_keys_fp8_rows.restype = None
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        I, L = ctypes.c_int, ctypes.c_int64
-        lib.oracle_threads.argtypes = []
-        lib.oracle_threads.restype = I
-        lib.oracle_visible.argtypes = [I, I, I]
-        lib.oracle_visible.restype = I
-        lib.oracle_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
-        lib.oracle_indexer_topk.restype = I
-        lib.oracle_indexer_topk_rows.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
-        lib.oracle_indexer_topk_rows.restype = I
-        lib.oracle_indexer_topk_rows_absmax.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P, P]
-        lib.oracle_indexer_topk_rows_absmax.restype = I
-        lib.oracle_score_keys_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, I, P]
-        lib.oracle_score_keys_rows.restype = None
-        lib.oracle_row_absmax_rows.argtypes = [P, P, P, I, I, I, I, P, I, P]
-        lib.oracle_row_absmax_rows.restype = None
-        lib.oracle_topk_scores.argtypes = [P, I, I, I, I, I, P, I, P, P]
-        lib.oracle_topk_scores.restype = I
-        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
-        lib.oracle_e4m3_decode.restype = ctypes.c_double
-        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
-        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
-        lib.oracle_quantize_e4m3_rows.argtypes = [P, L, I, P, P]
-        lib.oracle_quantize_e4m3_rows.restype = None
-        lib.oracle_indexer_topk_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, P, P]
-        lib.oracle_indexer_topk_fp8_rows.restype = I
-        lib.oracle_score_keys_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, I, P]
-        lib.oracle_score_keys_fp8_rows.restype = None
-        _lib = lib
+        _lib = declare(ctypes.CDLL(build()))
     return _lib
+
+
+class _Bound:
+    """The module's functions bound to another compiled copy of oracle.c."""
+
+    def __init__(self, path: str):
+        self._cdll = declare(ctypes.CDLL(path))
+
+    def __getattr__(self, name):
+        fn = _API[name]
+        return lambda *a, **kw: fn(*a, lib=self._cdll, **kw)
+
+
+def load_copy(path: str) -> "_Bound":
+    """The oracle API on a separately compiled copy of oracle.c (used by the
+    tests that plant mistakes in a copy and check that the pins catch them)."""
+    return _Bound(path)
+
+
+def _use(lib):
+    return lib if lib is not None else _load()
 
 
 def _c(a, dtype):
@@ -83,17 +109,17 @@ def _p(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def threads() -> int:
+def threads(lib=None) -> int:
     """OpenMP threads the oracle's row loops use."""
-    return _load().oracle_threads()
+    return _use(lib).oracle_threads()
 
 
-def visible(t: int, T: int, m: int) -> int:
+def visible(t: int, T: int, m: int, lib=None) -> int:
     """Number of compressed keys visible to query t (keys j with (j+1)m-1 <= t)."""
-    return _load().oracle_visible(int(t), int(T), int(m))
+    return _use(lib).oracle_visible(int(t), int(T), int(m))
 
 
-def indexer_topk(q, w, kc, m: int, k: int, rows=None):
+def indexer_topk(q, w, kc, m: int, k: int, rows=None, lib=None):
     """Oracle top-k from full tensors.
 
     q [B,S,H,D] uint16 (bf16 bits), w [B,S,H] float32, kc [B,T,D] uint16.
@@ -106,14 +132,14 @@ def indexer_topk(q, w, kc, m: int, k: int, rows=None):
     n = rows.size
     idx = np.empty((n, k), dtype=np.int32)
     sc = np.empty((n, k), dtype=np.float64)
-    rc = _load().oracle_indexer_topk(_p(q), _p(w), _p(kc), B, S, H, D, m, k, _p(rows), n, _p(idx),
-                                     _p(sc))
+    rc = _use(lib).oracle_indexer_topk(_p(q), _p(w), _p(kc), B, S, H, D, m, k, _p(rows), n,
+              _p(idx), _p(sc))
     if rc != 0:
         raise ValueError("oracle_indexer_topk: bad arguments")
     return idx, sc
 
 
-def indexer_topk_rows(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
+def indexer_topk_rows(q_rows, w_rows, kc, S: int, m: int, k: int, rows, lib=None):
     """Oracle top-k given only the listed queries' rows of q and w
     (q_rows [n,H,D], w_rows [n,H]); rows are their flat positions b*S+t."""
     q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
@@ -122,14 +148,14 @@ def indexer_topk_rows(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
     B = kc.shape[0]
     idx = np.empty((n, k), dtype=np.int32)
     sc = np.empty((n, k), dtype=np.float64)
-    rc = _load().oracle_indexer_topk_rows(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m, k,
-                                          _p(rows), n, _p(idx), _p(sc))
+    rc = _use(lib).oracle_indexer_topk_rows(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m, k,
+              _p(rows), n, _p(idx), _p(sc))
     if rc != 0:
         raise ValueError("oracle_indexer_topk_rows: bad arguments")
     return idx, sc
 
 
-def indexer_topk_rows_absmax(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
+def indexer_topk_rows_absmax(q_rows, w_rows, kc, S: int, m: int, k: int, rows, lib=None):
     """``indexer_topk_rows`` plus each row's max |score| over its visible keys."""
     q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
     rows = _c(rows, np.int64)
@@ -138,36 +164,37 @@ def indexer_topk_rows_absmax(q_rows, w_rows, kc, S: int, m: int, k: int, rows):
     idx = np.empty((n, k), dtype=np.int32)
     sc = np.empty((n, k), dtype=np.float64)
     amax = np.empty(n, dtype=np.float64)
-    rc = _load().oracle_indexer_topk_rows_absmax(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m, k,
-                                                 _p(rows), n, _p(idx), _p(sc), _p(amax))
+    rc = _use(lib).oracle_indexer_topk_rows_absmax(_p(q_rows), _p(w_rows), _p(kc), B, S, H, D, m,
+              k, _p(rows), n, _p(idx), _p(sc), _p(amax))
     if rc != 0:
         raise ValueError("oracle_indexer_topk_rows_absmax: bad arguments")
     return idx, sc, amax
 
 
-def score_keys_rows(q_rows, w_rows, kc, S: int, m: int, rows, js):
-    """fp64 scores of keys js[i, :] (entries < 0 give nan) for the listed queries."""
+def score_keys_rows(q_rows, w_rows, kc, S: int, m: int, rows, js, lib=None):
+    """fp64 scores of keys js[i, :] for the listed queries; keys a query cannot
+    see (j < 0 or j >= V_t) give nan."""
     q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
     rows, js = _c(rows, np.int64), _c(js, np.int32)
     n, H, D = q_rows.shape
     out = np.full(js.shape, np.nan, dtype=np.float64)
-    _load().oracle_score_keys_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n, _p(js),
-                                   js.shape[1], _p(out))
+    _use(lib).oracle_score_keys_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n,
+         _p(js), js.shape[1], _p(out))
     return out
 
 
-def row_absmax_rows(q_rows, w_rows, kc, S: int, m: int, rows):
+def row_absmax_rows(q_rows, w_rows, kc, S: int, m: int, rows, lib=None):
     """max over visible keys of |score| for each listed query."""
     q_rows, w_rows, kc = _c(q_rows, np.uint16), _c(w_rows, np.float32), _c(kc, np.uint16)
     rows = _c(rows, np.int64)
     n, H, D = q_rows.shape
     out = np.empty(n, dtype=np.float64)
-    _load().oracle_row_absmax_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n,
-                                   _p(out))
+    _use(lib).oracle_row_absmax_rows(_p(q_rows), _p(w_rows), _p(kc), S, H, D, m, _p(rows), n,
+         _p(out))
     return out
 
 
-def topk_scores(X, m: int, k: int, rows=None):
+def topk_scores(X, m: int, k: int, rows=None, lib=None):
     """Selection alone on given fp32 scores X [B,S,T].
     Returns (idx [n,k] int32, score [n,k] float32 carrying the input bit patterns)."""
     X = _c(X, np.float32)
@@ -176,55 +203,65 @@ def topk_scores(X, m: int, k: int, rows=None):
     n = rows.size
     idx = np.empty((n, k), dtype=np.int32)
     sc = np.empty((n, k), dtype=np.float32)
-    rc = _load().oracle_topk_scores(_p(X), B, S, T, m, k, _p(rows), n, _p(idx), _p(sc))
+    rc = _use(lib).oracle_topk_scores(_p(X), B, S, T, m, k, _p(rows), n, _p(idx), _p(sc))
     if rc != 0:
         raise ValueError("oracle_topk_scores: bad arguments")
     return idx, sc
 
 
-def e4m3_decode(code: int) -> float:
-    return _load().oracle_e4m3_decode(int(code))
+def e4m3_decode(code: int, lib=None) -> float:
+    return _use(lib).oracle_e4m3_decode(int(code))
 
 
-def e4m3_encode(y: float) -> int:
-    return _load().oracle_e4m3_encode(float(y))
+def e4m3_encode(y: float, lib=None) -> int:
+    return _use(lib).oracle_e4m3_encode(float(y))
 
 
-def quantize_e4m3_rows(x):
+def quantize_e4m3_rows(x, lib=None):
     """x [..., cols] uint16 bf16 bits -> (codes uint8 [..., cols], scale fp32 [...])."""
     x = _c(x, np.uint16)
     shp = x.shape
     x2 = x.reshape(-1, shp[-1])
     codes = np.empty(x2.shape, dtype=np.uint8)
     scale = np.empty(x2.shape[0], dtype=np.float32)
-    _load().oracle_quantize_e4m3_rows(_p(x2), x2.shape[0], x2.shape[1], _p(codes), _p(scale))
+    _use(lib).oracle_quantize_e4m3_rows(_p(x2), x2.shape[0], x2.shape[1], _p(codes), _p(scale))
     return codes.reshape(shp), scale.reshape(shp[:-1])
 
 
-def indexer_topk_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, k: int, rows):
+def indexer_topk_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, k: int, rows,
+                          lib=None):
     """Oracle top-k of the FP8 score (codes decoded exactly, scales applied in fp64).
 
     q8_rows [n,H,D] uint8, sq_rows [n,H] fp32, w_rows [n,H] fp32 for the listed
     queries; k8 [B,T,D] uint8, s_k [B,T] fp32."""
-    q8_rows, sq_rows, w_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32), _c(w_rows, np.float32)
+    q8_rows, sq_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32)
+    w_rows = _c(w_rows, np.float32)
     k8, s_k, rows = _c(k8, np.uint8), _c(s_k, np.float32), _c(rows, np.int64)
     n, H, D = q8_rows.shape
     B = k8.shape[0]
     idx = np.empty((n, k), dtype=np.int32)
     sc = np.empty((n, k), dtype=np.float64)
-    rc = _load().oracle_indexer_topk_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8),
-                                              _p(s_k), B, S, H, D, m, k, _p(rows), n, _p(idx),
-                                              _p(sc))
+    rc = _use(lib).oracle_indexer_topk_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8),
+              _p(s_k), B, S, H, D, m, k, _p(rows), n, _p(idx), _p(sc))
     if rc != 0:
         raise ValueError("oracle_indexer_topk_fp8_rows: bad arguments")
     return idx, sc
 
 
-def score_keys_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, rows, js):
-    q8_rows, sq_rows, w_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32), _c(w_rows, np.float32)
+def score_keys_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, rows, js, lib=None):
+    """FP8 scores of keys js[i, :] for the listed queries; keys a query cannot
+    see give nan."""
+    q8_rows, sq_rows = _c(q8_rows, np.uint8), _c(sq_rows, np.float32)
+    w_rows = _c(w_rows, np.float32)
     k8, s_k, rows, js = _c(k8, np.uint8), _c(s_k, np.float32), _c(rows, np.int64), _c(js, np.int32)
     n, H, D = q8_rows.shape
     out = np.full(js.shape, np.nan, dtype=np.float64)
-    _load().oracle_score_keys_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8), _p(s_k), S, H,
-                                       D, m, _p(rows), n, _p(js), js.shape[1], _p(out))
+    _use(lib).oracle_score_keys_fp8_rows(_p(q8_rows), _p(sq_rows), _p(w_rows), _p(k8), _p(s_k), S,
+         H, D, m, _p(rows), n, _p(js), js.shape[1], _p(out))
     return out
+
+
+_API = {name: globals()[name] for name in (
+    "threads", "visible", "indexer_topk", "indexer_topk_rows", "indexer_topk_rows_absmax",
+    "score_keys_rows", "row_absmax_rows", "topk_scores", "e4m3_decode", "e4m3_encode",
+    "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows")}

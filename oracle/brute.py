@@ -70,24 +70,29 @@ def e4m3_value(code: int) -> Fraction:
     return s * v
 
 
+def score_fp8(q8, s_q, w, k8, s_k, b: int, t: int, j: int) -> Fraction:
+    """Exact FP8 score of key j for query (b, t):
+    sum_h w * max(0, s_q[t,h] * s_k[j] * sum_d e4m3(q8) * e4m3(k8))."""
+    H, D = q8.shape[2], q8.shape[3]
+    s = Fraction(0)
+    for h in range(H):
+        dot = sum((e4m3_value(int(q8[b, t, h, d])) * e4m3_value(int(k8[b, j, d]))
+                   for d in range(D)), Fraction(0))
+        x = _f32(s_q[b, t, h]) * _f32(s_k[b, j]) * dot
+        s += _f32(w[b, t, h]) * max(Fraction(0), x)
+    return s
+
+
 def topk_fp8(q8, s_q, w, k8, s_k, m: int, k: int):
     """Exact-rational FP8 score top-k:
     score = sum_h w * max(0, s_q[t,h] * s_k[j] * sum_d e4m3(q8) * e4m3(k8))."""
-    B, S, H, D = q8.shape
+    B, S = q8.shape[:2]
     T = k8.shape[1]
     out_idx, out_sc = [], []
     for b in range(B):
         for t in range(S):
             V = visible_count(t, T, m)
-            pairs = []
-            for j in range(V):
-                s = Fraction(0)
-                for h in range(H):
-                    dot = sum((e4m3_value(int(q8[b, t, h, d])) * e4m3_value(int(k8[b, j, d]))
-                               for d in range(D)), Fraction(0))
-                    x = _f32(s_q[b, t, h]) * _f32(s_k[b, j]) * dot
-                    s += _f32(w[b, t, h]) * max(Fraction(0), x)
-                pairs.append((s, j))
+            pairs = [(score_fp8(q8, s_q, w, k8, s_k, b, t, j), j) for j in range(V)]
             pairs.sort(key=lambda p: (-p[0], p[1]))
             sel = pairs[:k]
             out_idx.append([j for _, j in sel] + [-1] * (k - len(sel)))

@@ -165,12 +165,14 @@ int oracle_indexer_topk_rows_absmax(const uint16_t* q_rows, const float* w_rows,
         const float* wr = w_rows + (int64_t)i * H;
         const uint16_t* kcb = kc + b * T * (int64_t)D;
         pair_t* p = (pair_t*)malloc(sizeof(pair_t) * (size_t)(V > 0 ? V : 1));
-        double mx = 0.0;
         for (int j = 0; j < V; j++) {
             p[j].s = oracle_score_row(qr, wr, kcb, H, D, j);
             p[j].j = j;
-            if (fabs(p[j].s) > mx) mx = fabs(p[j].s);
         }
+        /* the scale of the tolerance rule: largest |score| over the visible keys */
+        double mx = 0.0;
+        for (int j = 0; j < V; j++)
+            if (fabs(p[j].s) > mx) mx = fabs(p[j].s);
         qsort(p, (size_t)V, sizeof(pair_t), cmp_pair);
         for (int r = 0; r < k; r++) {
             out_idx[(int64_t)i * k + r] = r < V ? p[r].j : -1;
@@ -201,9 +203,11 @@ int oracle_indexer_topk(const uint16_t* q, const float* w, const uint16_t* kc, i
     return 0;
 }
 
-/* fp64 scores of keys js[i, 0..kk) (entries < 0 skipped, left untouched) for
- * listed queries given by their own rows; used to judge keys outside the
- * oracle's own top-k. */
+/* fp64 scores of keys js[i, 0..kk) for listed queries given by their own
+ * rows; used to judge keys outside the oracle's own top-k.  A key the query
+ * cannot see (j < 0 or j >= V_t) has no score: its entry is left untouched, so
+ * the caller's fill value (NaN) marks it, and no key past the batch's T is
+ * ever read. */
 void oracle_score_keys_rows(const uint16_t* q_rows, const float* w_rows, const uint16_t* kc, int S,
                             int H, int D, int m, const int64_t* rows, int n, const int32_t* js,
                             int kk, double* out) {
@@ -211,9 +215,10 @@ void oracle_score_keys_rows(const uint16_t* q_rows, const float* w_rows, const u
 #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < n; i++) {
         int64_t b = rows[i] / S;
+        int V = oracle_visible((int)(rows[i] % S), T, m);
         for (int r = 0; r < kk; r++) {
             int j = js[(int64_t)i * kk + r];
-            if (j < 0) continue;
+            if (j < 0 || j >= V) continue;
             out[(int64_t)i * kk + r] = oracle_score_row(q_rows + (int64_t)i * H * D,
                                                         w_rows + (int64_t)i * H,
                                                         kc + b * T * (int64_t)D, H, D, j);
@@ -395,6 +400,8 @@ int oracle_indexer_topk_fp8_rows(const uint8_t* q8_rows, const float* sq_rows,
     return 0;
 }
 
+/* FP8 scores of keys js[i, 0..kk) for listed queries given by their own rows;
+ * keys the query cannot see are left untouched, as in oracle_score_keys_rows. */
 void oracle_score_keys_fp8_rows(const uint8_t* q8_rows, const float* sq_rows, const float* w_rows,
                                 const uint8_t* k8, const float* sk, int S, int H, int D, int m,
                                 const int64_t* rows, int n, const int32_t* js, int kk,
@@ -403,9 +410,10 @@ void oracle_score_keys_fp8_rows(const uint8_t* q8_rows, const float* sq_rows, co
 #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < n; i++) {
         int64_t b = rows[i] / S;
+        int V = oracle_visible((int)(rows[i] % S), T, m);
         for (int r = 0; r < kk; r++) {
             int j = js[(int64_t)i * kk + r];
-            if (j < 0) continue;
+            if (j < 0 || j >= V) continue;
             out[(int64_t)i * kk + r] = oracle_score_row_fp8(
                 q8_rows + (int64_t)i * H * D, sq_rows + (int64_t)i * H, w_rows + (int64_t)i * H,
                 k8 + b * T * (int64_t)D, sk + b * T, H, D, j);

@@ -1,0 +1,157 @@
+"""The oracle's pins as one suite over an oracle API object.
+
+Each check ties an oracle function to something other than the oracle itself:
+the hand-worked values of tests/golden/hand_cases.json, exact rational
+arithmetic (oracle/brute.py) and the visibility rule written out.  The same
+suite runs on the built oracle (tests/test_oracle.py) and on copies with a
+planted mistake (tests/test_oracle_mutations.py), which it must reject.
+
+``o`` is the ``oracle`` module or ``oracle.load_copy(path)``.  Every check
+covers the functions the GPU parity tests and the smoke check call:
+indexer_topk, indexer_topk_rows, indexer_topk_rows_absmax (the rows, their
+scores and the max |score| that scales the tolerance rule), score_keys_rows
+(the score of a key outside the oracle's own top-k), row_absmax_rows and the
+FP8 pair indexer_topk_fp8_rows / score_keys_fp8_rows.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+from oracle import brute
+from tests import _golden
+
+
+def _same_scores(got, want) -> bool:
+    """fp64 scores equal, or both the same infinity (padding)."""
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    return bool(np.all((got == want) | (np.isinf(got) & np.isinf(want) & (got == want))))
+
+
+def _brute_scores(q, w, kc, m):
+    """Exact scores of every key for every query, as fp64 (None where the key
+    is not visible).  Values are dyadic with few bits, so fp64 holds them
+    exactly and fp64 equality is exact equality."""
+    B, S = q.shape[:2]
+    T = kc.shape[1]
+    out = np.full((B * S, T), np.nan)
+    for b in range(B):
+        for t in range(S):
+            for j in range(brute.visible_count(t, T, m)):
+                out[b * S + t, j] = float(brute.score(q, w, kc, b, t, j))
+    return out
+
+
+def _dyadic(seed, B, S, m, H, D):
+    """Values on the grid i/8, |i| <= 8: every fp64 product and sum of the
+    oracle is exact, and exact ties are frequent."""
+    g = np.random.default_rng(seed)
+    T = S // m
+    q = g.integers(-8, 9, size=(B, S, H, D)).astype(np.float32) / 8
+    kc = g.integers(-8, 9, size=(B, T, D)).astype(np.float32) / 8
+    w = g.integers(-8, 9, size=(B, S, H)).astype(np.float32) / 8
+    return synth.f32_to_bf16_bits(q), w, synth.f32_to_bf16_bits(kc)
+
+
+# (seed, B, S, m, H, D, k): two batches (batch offsets), rows t < m-1 that see
+# no key, rows that see fewer keys than k, m = 1
+DYADIC = [(11, 1, 12, 2, 3, 4, 4), (12, 2, 12, 3, 2, 3, 3), (13, 2, 8, 1, 2, 2, 5),
+          (14, 2, 16, 4, 3, 2, 2)]
+
+
+def check_hand_cases(o) -> None:
+    """The hand-worked rows through every row-producing entry, and the max
+    |score| of each row against the exact brute-force scores."""
+    for c in _golden.cases():
+        q, w, kc, m, k = c["q"], c["w"], c["kc"], c["m"], c["k"]
+        B, S = q.shape[:2]
+        rows = np.arange(B * S)
+        qr, wr = q.reshape(B * S, *q.shape[2:]), w.reshape(B * S, -1)
+        idx, sc = o.indexer_topk(q, w, kc, m, k)
+        assert np.array_equal(idx, c["idx"]) and _same_scores(sc, c["score"]), c["name"]
+        idx, sc = o.indexer_topk_rows(qr, wr, kc, S, m, k, rows)
+        assert np.array_equal(idx, c["idx"]) and _same_scores(sc, c["score"]), c["name"]
+        idx, sc, amax = o.indexer_topk_rows_absmax(qr, wr, kc, S, m, k, rows)
+        assert np.array_equal(idx, c["idx"]) and _same_scores(sc, c["score"]), c["name"]
+        exact = _brute_scores(q, w, kc, m)
+        want = np.max(np.abs(np.nan_to_num(exact, nan=0.0)), axis=1)
+        assert np.array_equal(amax, want), (c["name"], amax, want)
+
+
+def check_dyadic_brute_force(o) -> None:
+    """Every row function against exact rational arithmetic on dyadic inputs:
+    rows and scores, the visible-key max |score|, and the score of every key
+    j in [-1, T] (nan exactly where the key is not visible)."""
+    for seed, B, S, m, H, D, k in DYADIC:
+        q, w, kc = _dyadic(seed, B, S, m, H, D)
+        T = S // m
+        bi, bs = brute.topk(q, w, kc, m, k)
+        bi = np.array(bi)
+        bsf = np.array([[-np.inf if s is None else float(s) for s in r] for r in bs])
+        exact = _brute_scores(q, w, kc, m)
+        absmax = np.max(np.abs(np.nan_to_num(exact, nan=0.0)), axis=1)
+        rows = np.arange(B * S)
+        qr, wr = q.reshape(B * S, H, D), w.reshape(B * S, H)
+        oi, os_ = o.indexer_topk(q, w, kc, m, k)
+        assert np.array_equal(oi, bi) and _same_scores(os_, bsf), ("indexer_topk", seed)
+        oi, os_ = o.indexer_topk_rows(qr, wr, kc, S, m, k, rows)
+        assert np.array_equal(oi, bi) and _same_scores(os_, bsf), ("indexer_topk_rows", seed)
+        oi, os_, am = o.indexer_topk_rows_absmax(qr, wr, kc, S, m, k, rows)
+        assert np.array_equal(oi, bi) and _same_scores(os_, bsf), ("rows_absmax", seed)
+        assert np.array_equal(am, absmax), ("rows_absmax: absmax", seed, am, absmax)
+        assert np.array_equal(o.row_absmax_rows(qr, wr, kc, S, m, rows), absmax), ("row_absmax",
+                                                                                  seed)
+        # a reversed row subset: each row still finds its own batch and position
+        sub = rows[::-1][: max(1, rows.size // 2)]
+        oi, _, am = o.indexer_topk_rows_absmax(qr[sub], wr[sub], kc, S, m, k, sub)
+        assert np.array_equal(oi, bi[sub]) and np.array_equal(am, absmax[sub]), ("subset", seed)
+        # scores of given keys: every j in [-1, T], visible or not
+        js = np.broadcast_to(np.arange(-1, T + 1, dtype=np.int32), (B * S, T + 2))
+        js = np.where(js > T - 1, -1, js).astype(np.int32)
+        got = o.score_keys_rows(qr, wr, kc, S, m, rows, js)
+        want = np.where(js >= 0, exact[rows[:, None], np.maximum(js, 0)], np.nan)
+        same = (got == want) | (np.isnan(got) & np.isnan(want))
+        assert np.all(same), ("score_keys_rows", seed, got, want)
+
+
+def check_fp8_brute_force(o) -> None:
+    """The FP8 rows and key scores against exact rational arithmetic on the
+    decoded codes (codes and scales drawn directly, two batches)."""
+    g = np.random.default_rng(21)
+    B, S, m, H, D, k = 2, 12, 3, 2, 4, 3
+    T = S // m
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    q8 = g.choice(codes, size=(B, S, H, D))
+    k8 = g.choice(codes, size=(B, T, D))
+    s_q = (g.integers(1, 16, size=(B, S, H)) / 8).astype(np.float32)
+    s_k = (g.integers(1, 16, size=(B, T)) / 4).astype(np.float32)
+    w = (g.integers(-8, 9, size=(B, S, H)) / 8).astype(np.float32)
+    bi, bs = brute.topk_fp8(q8, s_q, w, k8, s_k, m, k)
+    rows = np.arange(B * S)
+    oi, os_ = o.indexer_topk_fp8_rows(q8.reshape(B * S, H, D), s_q.reshape(B * S, H),
+                                      w.reshape(B * S, H), k8, s_k, S, m, k, rows)
+    assert np.array_equal(oi, np.array(bi)), ("fp8 rows", oi, bi)
+    for r in range(B * S):
+        for c in range(k):
+            want = -np.inf if bs[r][c] is None else float(bs[r][c])
+            assert os_[r, c] == want or abs(os_[r, c] - want) <= 1e-14 * abs(want), ("fp8 score",
+                                                                                   r, c)
+    js = np.broadcast_to(np.arange(-1, T, dtype=np.int32), (B * S, T + 1)).copy()
+    got = o.score_keys_fp8_rows(q8.reshape(B * S, H, D), s_q.reshape(B * S, H),
+                                w.reshape(B * S, H), k8, s_k, S, m, rows, js)
+    for r in range(B * S):
+        b, t = divmod(r, S)
+        V = brute.visible_count(t, T, m)
+        for c, j in enumerate(js[r]):
+            if j < 0 or j >= V:
+                assert np.isnan(got[r, c]), ("fp8 key score of an invisible key", r, j)
+            else:
+                want = float(brute.score_fp8(q8, s_q, w, k8, s_k, b, t, int(j)))
+                assert abs(got[r, c] - want) <= 1e-14 * max(abs(want), 1e-300), ("fp8 key", r, j)
+
+
+def run_all(o) -> None:
+    check_hand_cases(o)
+    check_dyadic_brute_force(o)
+    check_fp8_brute_force(o)

@@ -165,3 +165,51 @@ def test_rejects_bad_arguments():
     q = np.zeros((1, 6, 1, 1), np.uint16)
     with pytest.raises(ValueError):
         oracle.indexer_topk(q, np.zeros((1, 6, 1), np.float32), np.zeros((1, 1, 1), np.uint16), 4, 1)
+
+
+# ---------------------------------------------------------------------------
+# the helpers the GPU parity tests and the smoke check call, pinned one by one
+# (tests/_pins.py; the mutation tests run the same checks on planted mistakes)
+
+from tests import _pins  # noqa: E402
+
+
+def test_pins_hand_cases_all_row_entries():
+    _pins.check_hand_cases(oracle)
+
+
+def test_pins_dyadic_brute_force_all_row_entries():
+    _pins.check_dyadic_brute_force(oracle)
+
+
+def test_pins_fp8_rows_and_key_scores_brute_force():
+    _pins.check_fp8_brute_force(oracle)
+
+
+def test_row_helpers_match_numpy_two_batches():
+    """Random bf16 inputs, two batches, rows t < m - 1 included: the max
+    |score| over visible keys and the scores of given keys (visible, -1 and
+    beyond the visible range) against an independent numpy fp64 computation."""
+    sh = synth.small(2, 256, 4, 8, 64, 16, seed=8, kc_kind="ar1")
+    q, w, kc = synth.gen_q(sh, 8), synth.gen_w(sh, 8), synth.gen_kc(sh, 8)
+    s = _numpy_scores(q, w, kc).reshape(2 * sh.S, sh.T)
+    g = np.random.default_rng(0)
+    rows = np.union1d(g.choice(2 * sh.S, 60, replace=False), [0, 1, 2, sh.S, sh.S + 2, 2 * sh.S - 1])
+    t = rows % sh.S
+    V = np.minimum(sh.T, (t + 1) // sh.m)
+    qr, wr = q.reshape(-1, sh.H, sh.D)[rows], w.reshape(-1, sh.H)[rows]
+    want_amax = np.array([np.abs(s[r, :v]).max() if v else 0.0 for r, v in zip(rows, V)])
+    oi, os_, amax = oracle.indexer_topk_rows_absmax(qr, wr, kc, sh.S, sh.m, sh.topk, rows)
+    np.testing.assert_allclose(amax, want_amax, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(oracle.row_absmax_rows(qr, wr, kc, sh.S, sh.m, rows), want_amax,
+                               rtol=1e-12, atol=0)
+    for i, (r, v) in enumerate(zip(rows, V)):
+        n = min(sh.topk, v)
+        np.testing.assert_allclose(os_[i, :n], np.sort(s[r, :v])[::-1][:n], rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(os_[i, :n], s[r, oi[i, :n]], rtol=1e-12, atol=1e-15)
+    js = g.integers(-1, sh.T, size=(rows.size, 40)).astype(np.int32)
+    got = oracle.score_keys_rows(qr, wr, kc, sh.S, sh.m, rows, js)
+    vis = (js >= 0) & (js < V[:, None])
+    assert np.all(np.isnan(got[~vis]))
+    np.testing.assert_allclose(got[vis], s[np.repeat(rows, 40).reshape(-1, 40)[vis], js[vis]],
+                               rtol=1e-12, atol=1e-15)

@@ -1,23 +1,26 @@
 """Plants plausible mistakes in a temporary copy of the oracle (on the CPU)
-and checks that the pins catch each one: a dropped ReLU, an off-by-one
-visibility rule, a reversed tie rule, a transposed operand, a wrong sign, a
-dropped head, a wrong padding value and an ascending sort."""
+and checks that the pins (tests/_pins.py) catch each one.
 
-import ctypes
+The mistakes cover the scoring definition (a dropped ReLU, a transposed
+operand, a wrong sign, a dropped head), the visibility rule, the order and
+padding of a row, and every helper the GPU parity tests and the smoke check
+call: the max |score| that scales the tolerance rule (no absolute value, an
+invisible key included, the wrong row's weights), the score of a given key
+(a dropped batch offset, no visibility check) and the FP8 scales."""
+
 import os
 import subprocess
 
-import numpy as np
 import pytest
 
-import synth
-from oracle import brute
-from tests import _golden
+import oracle
+from tests import _pins
 
 _SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle",
                     "oracle.c")
 
 MUTATIONS = {
+    # the score and the row
     "drop_relu": ("double r = dot > 0.0 ? dot : 0.0;", "double r = dot;"),
     "visibility_off_by_one": ("(v + 1) * m - 1 <= t", "(v + 1) * m - 1 < t"),
     "tie_rule_reversed": ("return (x->j < y->j) ? -1 : (x->j > y->j);\n}\n\nstatic int cmp_pairf",
@@ -34,6 +37,50 @@ MUTATIONS = {
                   "    return (x->j < y->j) ? -1 : (x->j > y->j);\n}\n\nstatic int cmp_pairf",
                   "    if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;\n"
                   "    return (x->j < y->j) ? -1 : (x->j > y->j);\n}\n\nstatic int cmp_pairf"),
+    # indexer_topk_rows_absmax: the rows and the tolerance scale
+    "absmax_no_abs": ("            if (fabs(p[j].s) > mx) mx = fabs(p[j].s);",
+                      "            if (p[j].s > mx) mx = p[j].s;"),
+    "absmax_over_all_T": (
+        "        for (int j = 0; j < V; j++)\n            if (fabs(p[j].s) > mx) mx = fabs(p[j].s);",
+        "        for (int j = 0; j < T; j++)\n"
+        "            if (fabs(oracle_score_row(qr, wr, kcb, H, D, j)) > mx)\n"
+        "                mx = fabs(oracle_score_row(qr, wr, kcb, H, D, j));"),
+    "absmax_row_weights_of_row_0": ("        const float* wr = w_rows + (int64_t)i * H;\n"
+                                    "        const uint16_t* kcb = kc + b * T * (int64_t)D;",
+                                    "        const float* wr = w_rows;\n"
+                                    "        const uint16_t* kcb = kc + b * T * (int64_t)D;"),
+    "absmax_rows_pad_zero": ("            out_score[(int64_t)i * k + r] = r < V ? p[r].s : -INFINITY;\n"
+                             "        }\n        out_absmax[i] = mx;",
+                             "            out_score[(int64_t)i * k + r] = r < V ? p[r].s : 0.0;\n"
+                             "        }\n        out_absmax[i] = mx;"),
+    "absmax_rows_no_batch_offset": ("        const uint16_t* kcb = kc + b * T * (int64_t)D;\n"
+                                    "        pair_t* p",
+                                    "        const uint16_t* kcb = kc;\n        pair_t* p"),
+    # score_keys_rows: the score of a given key
+    "score_keys_no_batch_offset": ("                                                        "
+                                   "kc + b * T * (int64_t)D, H, D, j);",
+                                   "                                                        "
+                                   "kc, H, D, j);"),
+    "score_keys_no_visibility": ("            if (j < 0 || j >= V) continue;\n"
+                                 "            out[(int64_t)i * kk + r] = oracle_score_row(",
+                                 "            if (j < 0) continue;\n"
+                                 "            out[(int64_t)i * kk + r] = oracle_score_row("),
+    "score_keys_weights_of_row_0": ("                                                        "
+                                    "w_rows + (int64_t)i * H,\n",
+                                    "                                                        "
+                                    "w_rows,\n"),
+    # row_absmax_rows
+    "row_absmax_over_all_T": ("        for (int j = 0; j < V; j++) {\n            double s = fabs(",
+                              "        for (int j = 0; j < T; j++) {\n            double s = fabs("),
+    # FP8
+    "fp8_key_scale_dropped": ("double skj = (double)skb[j];", "double skj = 1.0;"),
+    "fp8_query_scale_dropped": ("double x = (double)sqr[h] * skj * dot;", "double x = skj * dot;"),
+    "fp8_score_keys_no_batch_offset": ("                k8 + b * T * (int64_t)D, sk + b * T, H, D, j);",
+                                       "                k8, sk, H, D, j);"),
+    "fp8_score_keys_no_visibility": ("            if (j < 0 || j >= V) continue;\n"
+                                     "            out[(int64_t)i * kk + r] = oracle_score_row_fp8(",
+                                     "            if (j < 0) continue;\n"
+                                     "            out[(int64_t)i * kk + r] = oracle_score_row_fp8("),
 }
 
 
@@ -43,43 +90,15 @@ def _build(tmp_path, name, src):
     c.write_text(src)
     subprocess.check_call(["gcc", "-O1", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off",
                            "-o", str(so), str(c), "-lm"])
-    lib = ctypes.CDLL(str(so))
-    P, I = ctypes.c_void_p, ctypes.c_int
-    lib.oracle_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, I, P, P]
-    lib.oracle_indexer_topk.restype = I
-    return lib
+    return oracle.load_copy(str(so))
 
 
-def _run(lib, q, w, kc, m, k):
-    q = np.ascontiguousarray(q, np.uint16)
-    w = np.ascontiguousarray(w, np.float32)
-    kc = np.ascontiguousarray(kc, np.uint16)
-    B, S, H, D = q.shape
-    rows = np.arange(B * S, dtype=np.int64)
-    idx = np.empty((B * S, k), np.int32)
-    sc = np.empty((B * S, k), np.float64)
-    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
-    lib.oracle_indexer_topk(p(q), p(w), p(kc), B, S, H, D, m, k, p(rows), B * S, p(idx), p(sc))
-    return idx, sc
-
-
-def _pins_pass(lib) -> bool:
-    """The hand-worked cases and an exact-rational brute-force comparison."""
-    for c in _golden.cases():
-        idx, sc = _run(lib, c["q"], c["w"], c["kc"], c["m"], c["k"])
-        if not np.array_equal(idx, c["idx"]):
-            return False
-        same = (sc == c["score"]) | (np.isinf(sc) & np.isinf(c["score"]) & (sc == c["score"]))
-        if not np.all(same):
-            return False
-    g = np.random.default_rng(11)
-    B, S, m, H, D, k = 1, 12, 2, 3, 4, 4
-    q = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(B, S, H, D)).astype(np.float32) / 8)
-    kc = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(B, S // m, D)).astype(np.float32) / 8)
-    w = (g.integers(-8, 9, size=(B, S, H)).astype(np.float32) / 8)
-    bi, _ = brute.topk(q, w, kc, m, k)
-    idx, _ = _run(lib, q, w, kc, m, k)
-    return np.array_equal(idx, np.array(bi))
+def _pins_pass(o) -> bool:
+    try:
+        _pins.run_all(o)
+    except (AssertionError, ValueError):
+        return False
+    return True
 
 
 def test_unmutated_copy_passes(tmp_path):
@@ -90,6 +109,6 @@ def test_unmutated_copy_passes(tmp_path):
 def test_mutation_is_caught(tmp_path, name):
     src = open(_SRC).read()
     old, new = MUTATIONS[name]
-    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
-    lib = _build(tmp_path, name, src.replace(old, new, 1))
-    assert not _pins_pass(lib), f"pins did not catch mutation {name}"
+    assert src.count(old) == 1, f"mutation anchor for {name} found {src.count(old)} times"
+    o = _build(tmp_path, name, src.replace(old, new, 1))
+    assert not _pins_pass(o), f"pins did not catch mutation {name}"

@@ -2,13 +2,15 @@
 """Benchmark of the CSA lightning-indexer top-k step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload v4flash_s16k] [--key-chunk C] [--fp8]
+                    [--workload long_s256k] [--key-chunk C] [--fp8]
 
 A step is one pass of the whole hot path (score contraction on tensor cores,
 ReLU + weighted head sum, causal mask, streaming top-k and, when keys are
 chunked, the partition merge) over one batch of synthetic input.  The metric is
 causally visible query-key pairs per second; the JSON line also carries the
 achieved TFLOP/s against the measured bf16 tensor-core peak and the peak HBM.
+The default workload is the long-context step (S = 262,144, T = 65,536,
+H_I = 64, d_I = 128, top-2048), the largest that fits one GPU.
 
 With N > 1 (one process per GPU under torch.distributed.run) every rank runs
 its own independent problem of the same shape (weak scaling, no data-path
@@ -198,28 +200,29 @@ def run_reference(args, sh):
     return 0
 
 
+def library_plan(sh, args) -> dict:
+    """The plan the library runs for this workload and these options (host
+    query, no launch): tile shape, query blocks, launches per call."""
+    import streaming_top_lightning_b200 as stl
+
+    opts = stl.options(key_chunk=args.key_chunk, row_finish=args.row_finish,
+                       key_tile=args.key_tile, strip_slots=args.strip_slots)
+    return stl.plan(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, fp8=args.fp8, opts=opts)
+
+
 def kernel_launches_per_step(sh, args) -> int:
-    """Our kernel launches in one step, following the library's plan: per query
-    block a score launch and a finishing launch (the bucket-sort finish with
-    one key chunk, the merge with several), the row sort when topk > 512 and
-    the merge finished the rows, and the two quantiser launches of the FP8
-    path.  With rows finished in the fused kernel: one score launch (and the
-    row sort above 512).  Query blocks follow the scratch plan (512 MiB of
-    partial lists by default; 256/H_I queries per tile; partial lists of
-    ceil((K + K/4 + 64)/32)*32 keys per query and key chunk)."""
-    QT = 256 // sh.H
-    G = (sh.S + QT - 1) // QT
-    C = args.key_chunk if args.key_chunk else (sh.T + 127) // 128 * 128
-    nch = max(1, (sh.T + C - 1) // C)
-    L = (sh.topk + sh.topk // 4 + 64 + 31) // 32 * 32
-    fp8 = 2 if args.fp8 else 0
-    if nch == 1 and args.row_finish == 1:
-        return 1 + (1 if sh.topk > 512 else 0) + fp8
-    per_tile = sh.B * nch * QT * L * 8
-    tb = max(1, min(G, (512 << 20) // per_tile))
-    n_blocks = (G + tb - 1) // tb
-    sort = 1 if (nch > 1 and sh.topk > 512) else 0
-    return 2 * n_blocks + sort + fp8
+    """Our kernel launches in one step: the library's own count for one call
+    (a score launch per query block, the finishing launches, the row sort when
+    rows need it) plus, on the FP8 path, the two quantiser launches."""
+    return library_plan(sh, args)["launches"] + (2 if args.fp8 else 0)
+
+
+L2_BYTES = 126 * 10 ** 6
+
+
+def input_bytes(sh, fp8: bool) -> int:
+    q = sh.B * sh.S * sh.H * sh.D * (1 if fp8 else 2)
+    return q + sh.B * sh.S * sh.H * 4 + sh.B * sh.T * sh.D * (1 if fp8 else 2)
 
 
 def config_of(sh, args):
@@ -230,8 +233,10 @@ def config_of(sh, args):
             "strip_slots": args.strip_slots or "library choice",
             "score_path": "fp8-e4m3" if args.fp8 else "bf16",
             "pairs_per_step": causal_pairs(sh.S, sh.T, sh.m),
-            "l2": "inputs larger than L2: q alone is "
-                  f"{sh.B * sh.S * sh.H * sh.D * (1 if args.fp8 else 2) / 1e6:.0f} MB per step",
+            "l2": (f"inputs larger than L2: {input_bytes(sh, args.fp8) / 1e6:.0f} MB read per step"
+                   if input_bytes(sh, args.fp8) > L2_BYTES else
+                   f"L2 flushed between timed steps (inputs {input_bytes(sh, args.fp8) / 1e6:.0f} MB"
+                   " fit in L2; a 256 MB buffer is written outside each step's events)"),
             "parallelism": f"replicas x{args.gpus} (independent problems)"}
 
 
@@ -344,23 +349,32 @@ def run_native(args, sh):
         uuid = None
 
     K = args.steps
+    plan = library_plan(sh, args)
+    nblk = plan["query_blocks"]
+    # inputs that fit in L2 would be read from it by the next step: flush it
+    # between steps (outside the step's events) and time the steps alone
+    flush = input_bytes(sh, args.fp8) <= L2_BYTES
+    l2buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
-    # the library records the score kernel's own launch interval into these
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K)]
-    for a, b in kev:  # make sure the events exist before their handles are taken
-        a.record(stream)
-        b.record(stream)
+    # the library records each query block's score-kernel launch into these,
+    # so the score kernel's own time excludes the finishing launches
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nblk)] for _ in range(K)]
+    for lst in kev:  # make sure the events exist before their handles are taken
+        for e in lst:
+            e.record(stream)
     torch.cuda.synchronize()
-    kopts = [stl.options(key_chunk=args.key_chunk, score_events=e, row_finish=args.row_finish,
-                         key_tile=args.key_tile, strip_slots=args.strip_slots) for e in kev]
+    kopts = [stl.options(key_chunk=args.key_chunk, score_event_list=lst,
+                         row_finish=args.row_finish, key_tile=args.key_tile,
+                         strip_slots=args.strip_slots) for lst in kev]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
         barrier()
         torch.cuda.synchronize()
         t_start.record(stream)
         for i in range(K):
+            if flush:
+                l2buf.fill_(i & 0xFF)
             timed["opts"] = kopts[i]
             ev[i][0].record(stream)
             step()
@@ -372,15 +386,19 @@ def run_native(args, sh):
     rc = stl.device_error()
     if rc != 0:
         raise RuntimeError(f"device error {rc} in the timed region")
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if flush:
+        total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev))
+    else:
+        total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    # score-kernel device time per step: the sum of its query blocks' launches
+    launch_ms = statistics.mean(sum(lst[2 * b].elapsed_time(lst[2 * b + 1]) for b in range(nblk))
+                                for lst in kev)
 
     # end to end through the public API: host -> device inputs, the call,
     # device -> host result, every step
     if args.no_e2e:
         return finish(args, sh, ranks, P, K, total_ms, launch_ms, None, None, None, None,
-                      peak_alloc, free0, free1, clk)
+                      peak_alloc, free0, free1, clk, plan)
     idx_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32).pin_memory()
     score_h = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32).pin_memory()
     qe = torch.empty_like(q_h, device=dev)
@@ -419,11 +437,11 @@ def run_native(args, sh):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     assert stl.device_error() == 0
     return finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h,
-                  peak_alloc, free0, free1, clk)
+                  peak_alloc, free0, free1, clk, plan)
 
 
 def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, peak_alloc,
-           free0, free1, clk):
+           free0, free1, clk, plan):
     world, rank, dist = ranks.world, ranks.rank, ranks.dist
     flops_per_pair = 2 * sh.H * sh.D
     ms_per_step = total_ms / K
@@ -434,7 +452,7 @@ def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, pea
     peak_tf = float(peaks["bf16_tflops"]) * (2.0 if args.fp8 else 1.0)
     tflops_step = flops_launch / (ms_per_step / 1e3) / 1e12
     traffic = traffic_record(sh.name, args.fp8)
-    launches_per_step = kernel_launches_per_step(sh, args)
+    launches_per_step = plan["launches"] + (2 if args.fp8 else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -450,8 +468,14 @@ def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, pea
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": traffic,
                      "kernel": "k_score_topk", "peak_source": f"{peak_src} bf16_tflops (burst)"
                      + (" x2 nominal fp8/bf16 ratio" if args.fp8 else ""),
-                     "algorithmic_flops_per_launch": flops_launch,
-                     "avg_launch_ms": launch_ms},
+                     "algorithmic_flops_per_step": flops_launch,
+                     "score_kernel_ms_per_step": launch_ms,
+                     "score_launches_per_step": plan["query_blocks"],
+                     "avg_launch_ms": launch_ms / plan["query_blocks"],
+                     "timing": "sum over the step's query blocks of CUDA events recorded by "
+                               "the library around each score-kernel launch"},
+        "plan": {k: plan[k] for k in ("queries_per_tile", "mma_n", "key_tile", "stages",
+                                      "strip_slots", "pool_keys", "query_blocks", "launches")},
         "e2e": None if e2e_ms is None else {
             "value": ranks.job_value(P * sh.B, e2e_ms / Ke), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -474,10 +498,10 @@ def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, pea
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="v4flash_s16k", choices=sorted(synth.SHAPES))
+    ap.add_argument("--workload", default="long_s256k", choices=sorted(synth.SHAPES))
     ap.add_argument("--key-chunk", type=int, default=0)
     ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
                     help="1: rows finished in the fused kernel; 2: by the merge kernel; "

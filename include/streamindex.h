@@ -95,7 +95,43 @@ typedef struct si_options {
   int strip_slots;      /* score strips in flight between the epilogue and
                            the selection warps: 2 to 4; 0 = the library's
                            choice.  Default 0. */
+  void** score_event_list; /* optional array of score_event_count
+                           cudaEvent_t (NULL = none): the call records
+                           [2i] on `stream` just before the score-kernel
+                           launch of query block i and [2i+1] just after it,
+                           for i < score_event_count / 2, so the score
+                           kernel's own device time excludes the finishing
+                           launches between query blocks (si_plan_info
+                           .query_blocks gives the count needed).  The
+                           events stay owned by the caller. */
+  int score_event_count;
+  int plan_heads;       /* si_topk_scores only: when > 0, select with the
+                           fused score kernel's plan for H_I = plan_heads,
+                           d_I = plan_dim and the bf16 (plan_fp8 = 0) or FP8
+                           (1) path (queries per tile, keys per strip, pool
+                           room, partial-list length), so the bit-exact test
+                           entry runs exactly the selection the indexer runs
+                           for that shape.  0 = the test entry's own plan
+                           (4 queries, 1024-key strips).  Default 0. */
+  int plan_dim;
+  int plan_fp8;
 } si_options;
+
+/* The plan of one indexer call, as the library would run it. */
+typedef struct si_plan_info {
+  int queries_per_tile;   /* queries of one tensor-core tile (mma_n / H_I) */
+  int mma_n;              /* MMA N: (query, head) columns of a tile, 128 or 256 */
+  int key_tile;           /* keys per score strip handed to the selection warps */
+  int stages;             /* key-tile pipeline stages in shared memory */
+  int strip_slots;        /* score strips in flight */
+  int pool_keys;          /* candidate-pool entries per query */
+  int partial_len;        /* candidates per query and key chunk in the scratch lists */
+  int key_chunks;         /* key chunks of the longest query tile */
+  int query_blocks;       /* query blocks, i.e. score-kernel launches of one call */
+  int launches;           /* kernel launches of one call */
+  size_t workspace_bytes; /* device workspace of si_indexer_topk_ex for this plan */
+  size_t smem_bytes;      /* dynamic shared memory of one score-kernel CTA */
+} si_plan_info;
 
 /* ---- the indexer step ------------------------------------------------ */
 
@@ -115,6 +151,21 @@ int si_indexer_topk(const void* q, const float* w, const void* kc, int B, int S,
 /* Bytes of device workspace si_indexer_topk_ex needs for this problem. */
 int si_indexer_topk_workspace_size(int B, int S, int H_I, int d_I, int m, int topk,
                                    const si_options* opt, size_t* bytes);
+
+/*
+ * si_indexer_topk_plan: the plan si_indexer_topk_ex (fp8 = 0) or
+ * si_indexer_topk_fp8 (fp8 = 1) would run for this problem and these options:
+ * tile shape, shared-memory plan, key chunks, query blocks and the number of
+ * kernel launches of one call (the FP8 quantiser launches, which are separate
+ * calls, are not counted).  Host only, nothing is launched.  The plan is made
+ * for the current device; on a host with no usable CUDA device it is made for
+ * the sm_100 limits (227 KB of shared memory per CTA).  Errors as the
+ * workspace-size query, plus SI_ERR_TOPK when the selection pools of this
+ * topk do not fit the shape's tile and SI_ERR_OPTIONS for a key_tile above
+ * the largest strip the tile allows.
+ */
+int si_indexer_topk_plan(int B, int S, int H_I, int d_I, int m, int topk, int fp8,
+                         const si_options* opt, si_plan_info* out);
 
 /* As si_indexer_topk, with options and a caller-provided device workspace of
  * ws_bytes (at least what si_indexer_topk_workspace_size reports). */

@@ -16,11 +16,11 @@ from __future__ import annotations
 import ctypes
 
 from . import _lib
-from ._lib import SiOptions, StreamIndexError  # noqa: F401
+from ._lib import SiOptions, SiPlanInfo, StreamIndexError  # noqa: F401
 
 __all__ = [
-    "indexer_topk", "indexer_topk_noalloc", "indexer_topk_fp8", "quantize_fp8_rows", "topk_scores", "workspace_size",
-    "device_error", "options", "version", "StreamIndexError",
+    "indexer_topk", "indexer_topk_noalloc", "indexer_topk_fp8", "quantize_fp8_rows", "topk_scores",
+    "workspace_size", "plan", "device_error", "options", "version", "StreamIndexError",
 ]
 
 
@@ -52,22 +52,34 @@ def _need(t, dtype, ndim, name):
 
 def options(key_chunk: int = 0, scratch_mb: int = 0, grid_ctas: int = 0, timeout_ms: int = 0,
             debug_flags: int = 0, score_events=None, row_finish: int = 0,
-            key_tile: int = 0, strip_slots: int = 0) -> SiOptions:
+            key_tile: int = 0, strip_slots: int = 0, score_event_list=None,
+            plan_heads: int = 0, plan_dim: int = 0, plan_fp8: int = 0) -> SiOptions:
     """Tuning knobs of include/streamindex.h.  ``score_events`` is an optional
     pair of ``torch.cuda.Event(enable_timing=True)`` that the call records around
-    its score-kernel launches (on the call's stream).  ``row_finish``: 1 = rows
-    finished in the fused kernel, 2 = by the merge kernel, 0 = the library's
-    choice.  ``key_tile``: keys per score strip (128, 256, 512; 0 = the
-    library's choice); ``strip_slots``: score strips in flight (2..4; 0 = the
-    library's choice)."""
+    its score-kernel launches (on the call's stream); ``score_event_list`` a
+    list of such events, recorded in pairs around each query block's score
+    launch.  ``row_finish``: 1 = rows finished in the fused kernel, 2 = by the
+    merge kernel, 0 = the library's choice.  ``key_tile``: keys per score strip
+    (128 .. 1024; 0 = the library's choice); ``strip_slots``: score strips in
+    flight (2..4; 0 = the library's choice).  ``plan_heads``/``plan_dim``/
+    ``plan_fp8``: make ``topk_scores`` select with the fused kernel's plan for
+    that indexer shape."""
     o = SiOptions(key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags)
     o.row_finish = row_finish
     o.key_tile = key_tile
     o.strip_slots = strip_slots
+    o.plan_heads = plan_heads
+    o.plan_dim = plan_dim
+    o.plan_fp8 = plan_fp8
     if score_events is not None:
         a, b = score_events
         o.score_events[0] = a.cuda_event
         o.score_events[1] = b.cuda_event
+    if score_event_list:
+        arr = (ctypes.c_void_p * len(score_event_list))(*[e.cuda_event for e in score_event_list])
+        o._event_array = arr  # keep the array alive as long as the options
+        o.score_event_list = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+        o.score_event_count = len(score_event_list)
     return o
 
 
@@ -83,6 +95,19 @@ def workspace_size(B: int, S: int, H: int, D: int, m: int, topk: int, opts: SiOp
                                                   ctypes.byref(opts) if opts else None,
                                                   ctypes.byref(n)))
     return n.value
+
+
+def plan(B: int, S: int, H: int, D: int, m: int, topk: int, fp8: bool = False,
+         opts: SiOptions | None = None) -> dict:
+    """The plan the library would run for this problem (si_indexer_topk_plan):
+    tile shape, shared-memory plan, key chunks, query blocks and launches."""
+    info = SiPlanInfo()
+    lib = _lib.load()
+    _lib.check("si_indexer_topk_plan",
+               lib.si_indexer_topk_plan(B, S, H, D, m, topk, 1 if fp8 else 0,
+                                        ctypes.byref(opts) if opts else None,
+                                        ctypes.byref(info)))
+    return info.as_dict()
 
 
 def _outputs(B, S, topk, device, out):

@@ -22,7 +22,7 @@ STATUS = {
 EXPORTS = [
     "si_indexer_topk", "si_indexer_topk_workspace_size", "si_indexer_topk_ex",
     "si_indexer_topk_fp8", "si_quantize_fp8_rows", "si_topk_scores", "si_status_string",
-    "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc",
+    "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc", "si_indexer_topk_plan",
 ]
 
 
@@ -31,7 +31,21 @@ class SiOptions(ctypes.Structure):
                 ("grid_ctas", ctypes.c_int), ("timeout_ms", ctypes.c_int),
                 ("debug_flags", ctypes.c_int), ("score_events", ctypes.c_void_p * 2),
                 ("row_finish", ctypes.c_int), ("key_tile", ctypes.c_int),
-                ("strip_slots", ctypes.c_int)]
+                ("strip_slots", ctypes.c_int), ("score_event_list", ctypes.POINTER(ctypes.c_void_p)),
+                ("score_event_count", ctypes.c_int), ("plan_heads", ctypes.c_int),
+                ("plan_dim", ctypes.c_int), ("plan_fp8", ctypes.c_int)]
+
+
+class SiPlanInfo(ctypes.Structure):
+    _fields_ = [("queries_per_tile", ctypes.c_int), ("mma_n", ctypes.c_int),
+                ("key_tile", ctypes.c_int), ("stages", ctypes.c_int),
+                ("strip_slots", ctypes.c_int), ("pool_keys", ctypes.c_int),
+                ("partial_len", ctypes.c_int), ("key_chunks", ctypes.c_int),
+                ("query_blocks", ctypes.c_int), ("launches", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t), ("smem_bytes", ctypes.c_size_t)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 
 class StreamIndexError(RuntimeError):
@@ -56,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.si_indexer_topk.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P]
     lib.si_indexer_topk_noalloc.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P]
     lib.si_indexer_topk_workspace_size.argtypes = [I, I, I, I, I, I, OP, ctypes.POINTER(Z)]
+    lib.si_indexer_topk_plan.argtypes = [I, I, I, I, I, I, I, OP, ctypes.POINTER(SiPlanInfo)]
     lib.si_indexer_topk_ex.argtypes = [P, P, P, I, I, I, I, I, I, P, P, OP, P, Z, P]
     lib.si_indexer_topk_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, OP, P, Z, P]
     lib.si_quantize_fp8_rows.argtypes = [P, L, I, P, P, P]

@@ -69,6 +69,20 @@ int dev_info(DevInfo** out) {
   return SI_OK;
 }
 
+// Shared memory and SM count to plan with: the current device's, or the
+// sm_100 limits (227 KB of opt-in shared memory per CTA, 148 SMs) on a host
+// with no usable device.  Used by the plan query only.
+void plan_limits(int* max_smem, int* sms) {
+  DevInfo* dev = nullptr;
+  if (dev_info(&dev) == SI_OK) {
+    *max_smem = dev->max_smem;
+    *sms = dev->sms;
+  } else {
+    *max_smem = 227 * 1024;
+    *sms = 148;
+  }
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -91,11 +105,19 @@ struct Opts {
   int key_chunk, scratch_mb, grid_ctas, timeout_ms, debug_flags, row_finish, key_tile,
       strip_slots;
   cudaEvent_t ev_begin, ev_end;
+  cudaEvent_t* ev_list;  // [2i], [2i+1] around query block i's score launch
+  int ev_count;
+  int plan_heads, plan_dim, plan_fp8;  // si_topk_scores: the fused kernel's plan
 };
 
 int read_opts(const si_options* o, Opts* out) {
-  Opts d{0, 512, 0, 2000, 0, 0, 0, 0, nullptr, nullptr};
+  Opts d{0, 512, 0, 2000, 0, 0, 0, 0, nullptr, nullptr, nullptr, 0, 0, 0, 0};
   if (o) {
+    d.ev_list = reinterpret_cast<cudaEvent_t*>(o->score_event_list);
+    d.ev_count = o->score_event_list ? o->score_event_count : 0;
+    d.plan_heads = o->plan_heads;
+    d.plan_dim = o->plan_dim;
+    d.plan_fp8 = o->plan_fp8;
     d.row_finish = o->row_finish;
     d.key_tile = o->key_tile;
     d.strip_slots = o->strip_slots;
@@ -111,7 +133,11 @@ int read_opts(const si_options* o, Opts* out) {
       d.row_finish < 0 || d.row_finish > 2 ||
       !(d.key_tile == 0 || d.key_tile == 128 || d.key_tile == 256 || d.key_tile == 512 ||
         d.key_tile == 1024) ||
-      d.strip_slots < 0 || d.strip_slots == 1 || d.strip_slots > 4)
+      d.strip_slots < 0 || d.strip_slots == 1 || d.strip_slots > 4 || d.ev_count < 0 ||
+      !(d.plan_heads == 0 || d.plan_heads == 8 || d.plan_heads == 16 || d.plan_heads == 32 ||
+        d.plan_heads == 64) ||
+      (d.plan_heads > 0 && !(d.plan_dim == 64 || d.plan_dim == 128)) || d.plan_fp8 < 0 ||
+      d.plan_fp8 > 1)
     return SI_ERR_OPTIONS;
   *out = d;
   return SI_OK;
@@ -174,6 +200,18 @@ bool rows_come_sorted(const Plan& pl, int K) {
   return rows_sorted_in_warp(K) || (!pl.final_rows && pl.nch_max == 1);
 }
 
+// Kernel launches of one call: a score launch per query block, a finishing
+// launch after each unless the fused kernel finishes the rows, and the row
+// sort when the rows do not come out sorted.
+int plan_launches(const Plan& pl, int K) {
+  return pl.n_blocks * (pl.final_rows ? 1 : 2) + (rows_come_sorted(pl, K) ? 0 : 1);
+}
+
+int plan_status(const ScorePlan& sp) {
+  if (sp.ok) return SI_OK;
+  return sp.err == 2 ? SI_ERR_OPTIONS : SI_ERR_TOPK;
+}
+
 int check_common(int B, int S, int m, int topk) {
   if (B < 1 || S < 1 || m < 1 || S % m != 0) return SI_ERR_DIM;
   if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
@@ -204,7 +242,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
   const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile, o.strip_slots);
-  if (!sp_plan.ok) return SI_ERR_TOPK;  // the selection pools of this topk do not fit
+  if ((rc = plan_status(sp_plan))) return rc;  // pools of this topk do not fit, or key_tile
   const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
   if (!aligned16(ws)) return SI_ERR_ALIGN;
@@ -256,8 +294,12 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     if (grid < 1) grid = 1;
     if (blk == 0 && o.ev_begin && cudaEventRecord(o.ev_begin, stream) != cudaSuccess)
       return SI_ERR_CUDA;
+    const bool blk_ev = o.ev_list && 2 * blk + 1 < o.ev_count;
+    if (blk_ev && cudaEventRecord(o.ev_list[2 * blk], stream) != cudaSuccess) return SI_ERR_CUDA;
     if (launch_score_topk(fp8, D, H, sp_plan.nq, tm_q, tm_kc, p, grid, sp_plan.smem, stream) !=
         cudaSuccess)
+      return SI_ERR_CUDA;
+    if (blk_ev && cudaEventRecord(o.ev_list[2 * blk + 1], stream) != cudaSuccess)
       return SI_ERR_CUDA;
     if (blk + 1 == pl.n_blocks && o.ev_end && cudaEventRecord(o.ev_end, stream) != cudaSuccess)
       return SI_ERR_CUDA;
@@ -365,6 +407,38 @@ int si_indexer_topk_workspace_size(int B, int S, int H_I, int d_I, int m, int to
   return workspace_for(false, S, B, H_I, d_I, m, topk, opt, bytes);
 }
 
+int si_indexer_topk_plan(int B, int S, int H_I, int d_I, int m, int topk, int fp8,
+                         const si_options* opt, si_plan_info* out) {
+  if (!out) return SI_ERR_NULL;
+  int rc = check_common(B, S, m, topk);
+  if (rc) return rc;
+  if (!(H_I == 8 || H_I == 16 || H_I == 32 || H_I == 64) || !(d_I == 64 || d_I == 128))
+    return SI_ERR_DIM;
+  if (fp8 < 0 || fp8 > 1) return SI_ERR_OPTIONS;
+  Opts o;
+  if ((rc = read_opts(opt, &o))) return rc;
+  int max_smem = 0, sms = 0;
+  plan_limits(&max_smem, &sms);
+  const ScorePlan sp = plan_score(fp8 != 0, d_I, H_I, topk, max_smem, o.key_tile, o.strip_slots);
+  if ((rc = plan_status(sp))) return rc;
+  const Plan pl = make_plan(B, S, S / m, topk, sp.QT, o);
+  si_plan_info r{};
+  r.queries_per_tile = sp.QT;
+  r.mma_n = sp.nq;
+  r.key_tile = sp.CS;
+  r.stages = sp.nst;
+  r.strip_slots = sp.nslot;
+  r.pool_keys = sp.cap;
+  r.partial_len = pl.L;
+  r.key_chunks = pl.nch_max;
+  r.query_blocks = pl.n_blocks;
+  r.launches = plan_launches(pl, topk);
+  r.workspace_bytes = pl.ws_bytes();
+  r.smem_bytes = sp.smem;
+  *out = r;
+  return SI_OK;
+}
+
 int si_indexer_topk_ex(const void* q, const float* w, const void* kc, int B, int S, int H_I,
                        int d_I, int m, int topk, int32_t* out_idx, float* out_score,
                        const si_options* opt, void* workspace, size_t ws_bytes, void* stream) {
@@ -424,8 +498,19 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int QT = 4, CS = 1024;
-  const int cap = ((std::max(topk + 64, 2 * topk) + 31) / 32) * 32;
+  int QT = 4, CS = 1024;
+  int cap = ((std::max(topk + 64, 2 * topk) + 31) / 32) * 32;
+  if (o.plan_heads > 0) {
+    // the fused kernel's selection plan for that shape: same queries per
+    // tile, strip length and pool room, hence the same selection steps
+    const ScorePlan fp = plan_score(o.plan_fp8 != 0, o.plan_dim, o.plan_heads, topk,
+                                    dev->max_smem, o.key_tile, o.strip_slots);
+    if ((rc = plan_status(fp))) return rc;
+    QT = fp.QT;
+    CS = fp.CS;
+    cap = fp.cap;
+    if (topk_scores_smem_bytes(QT, cap, CS) > (size_t)dev->max_smem) return SI_ERR_TOPK;
+  }
   // the selection-only path sees T keys per row; m still sets visibility
   const Plan pl = make_plan(B, S, T, topk, QT, o);
   const size_t bytes = pl.ws_bytes();

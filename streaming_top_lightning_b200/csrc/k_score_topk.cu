@@ -546,6 +546,9 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap&
   return cudaErrorInvalidValue;
 }
 
+// Largest score strip (keys per query) for QT queries per tile.
+static int strip_max(int QT);
+
 // Shared-memory plan for one MMA width NQ: the query tile (NQ rows), NST
 // key-tile stages, a ring of NSL score strips of CS keys per query (cs_req and
 // nsl_req > 0 fix them), the selection pools (cap keys per query) and the small
@@ -566,7 +569,7 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
                        sizeof(ScoreCtlSmem);
   const int cap_min = ((K + 64 + 31) / 32) * 32;
   const int cap_max = std::max(cap_min, 4 * K);
-  const int cs_max = std::min(1024, std::max(128, 4096 / QT));
+  const int cs_max = strip_max(QT);
   // key-tile stages wanted: a full-width tile's MMA (1024 cycles at the
   // dense rate) hides a tile load from L2 with two stages; a half-width
   // tile's takes half as long and needs three
@@ -613,11 +616,15 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
 // (N = 128) halves the queries per tile and so doubles each query's pool,
 // which keeps pruning rare, at the price of reading each key tile from shared
 // memory for half as many columns.
+static int strip_max(int QT) { return std::min(1024, std::max(128, 4096 / QT)); }
+
 ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req) {
-  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
+  ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
   if (full.ok && full.cap >= (3 * K) / 2) return full;
-  const ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
+  ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
   if (half.ok && (!full.ok || half.cap > full.cap)) return half;
+  if (!full.ok)
+    full.err = (cs_req > strip_max(kN / H) && cs_req > strip_max(kN / 2 / H)) ? 2 : 1;
   return full;
 }
 

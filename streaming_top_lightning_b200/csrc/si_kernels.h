@@ -34,6 +34,8 @@ struct ScorePlan {
   int cap;       // selection pool entries per query
   size_t smem;   // dynamic shared memory bytes
   bool ok;
+  int err;       // when !ok: 1 = the pools of this topk do not fit, 2 = cs_req
+                 // above the largest strip either tile width allows
 };
 
 // cs_req: keys per score strip (128 .. 1024), nsl_req: strip ring slots

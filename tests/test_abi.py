@@ -108,3 +108,52 @@ def test_strip_options_validated(lib):
         assert (rc == 0) == ok, (kt, ss, rc)
         if not ok:
             assert rc == -8
+
+
+def _plan(lib, B, S, H, D, m, k, fp8=0, opts=None):
+    info = _lib.SiPlanInfo()
+    rc = lib.si_indexer_topk_plan(B, S, H, D, m, k, fp8, ctypes.byref(opts) if opts else None,
+                                  ctypes.byref(info))
+    return rc, info
+
+
+def test_plan_query(lib):
+    # host-only: on a machine without a GPU the plan is made for the sm_100
+    # limits, so these hold on the CPU and on a B200 alike
+    rc, p = _plan(lib, 1, 16384, 64, 128, 4, 512)
+    assert rc == 0
+    assert (p.queries_per_tile, p.mma_n, p.key_chunks, p.query_blocks, p.launches) == (4, 256, 1,
+                                                                                        1, 2)
+    assert p.pool_keys >= 512 + 64 and p.partial_len == 704
+    assert p.smem_bytes <= 227 * 1024
+    rc, n = _ws(lib, 1, 16384, 64, 128, 4, 512)
+    assert rc == 0 and p.workspace_bytes <= n
+    # top-2048 takes the half-width tile (two queries per tile at H_I = 64);
+    # its 2624-key lists at S = 262,144 need eleven query blocks
+    rc, p = _plan(lib, 1, 262144, 64, 128, 4, 2048)
+    assert rc == 0 and (p.queries_per_tile, p.mma_n, p.query_blocks, p.launches) == (2, 128, 11,
+                                                                                      22)
+    assert p.pool_keys >= 3 * 2048 // 2
+    # chunked: score + merge per block and the row sort above k = 512
+    o = _lib.SiOptions(1024, 0, 0, 0, 0)
+    rc, p = _plan(lib, 1, 32768, 64, 128, 4, 1024, opts=o)
+    assert rc == 0 and (p.key_chunks, p.query_blocks, p.launches) == (8, 6, 13)
+    # errors: topk above the shape's limit, a strip above the tile's limit,
+    # bad dims and a bad fp8 flag
+    assert _plan(lib, 1, 4096, 8, 128, 4, 1024)[0] == -3
+    o = _lib.SiOptions(0, 0, 0, 0, 0)
+    o.key_tile = 1024
+    assert _plan(lib, 1, 4096, 8, 128, 4, 64, opts=o)[0] == -8   # 32 queries: strips <= 128
+    assert _plan(lib, 1, 4096, 64, 128, 4, 64, opts=o)[0] == 0
+    assert _plan(lib, 1, 4095, 64, 128, 4, 64)[0] == -2
+    assert _plan(lib, 1, 4096, 64, 128, 4, 64, fp8=2)[0] == -8
+    assert lib.si_indexer_topk_plan(1, 4096, 64, 128, 4, 64, 0, None, None) == -1
+
+
+def test_plan_hint_options_validated(lib):
+    for heads, dim, fp8, ok in [(0, 0, 0, True), (64, 128, 0, True), (8, 64, 1, True),
+                                (48, 128, 0, False), (64, 96, 0, False), (64, 128, 2, False)]:
+        o = _lib.SiOptions(0, 0, 0, 0, 0)
+        o.plan_heads, o.plan_dim, o.plan_fp8 = heads, dim, fp8
+        rc, _ = _ws(lib, 1, 16384, 64, 128, 4, 512, o)
+        assert (rc == 0) == ok, (heads, dim, fp8, rc)

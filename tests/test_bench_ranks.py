@@ -79,10 +79,11 @@ def test_reference_arm_idle_on_other_ranks(monkeypatch, capsys):
 
 
 def test_launch_count_follows_the_plan():
-    # one key chunk: a score and a bucket-sort finishing launch per query
-    # block, no row sort whatever k; several chunks: score + merge per block
-    # and the row sort above k = 512; FP8 adds the two quantiser launches;
-    # rows finished in the fused kernel: one launch (and the sort above 512)
+    # bench.py counts launches from the library's own plan query: one key
+    # chunk gives a score and a bucket-sort finishing launch per query block,
+    # no row sort whatever k; several chunks give score + merge per block and
+    # the row sort above k = 512; FP8 adds the two quantiser launches; rows
+    # finished in the fused kernel take one launch (and the sort above 512)
     sys.path.insert(0, ROOT)
     import bench
     import synth
@@ -90,12 +91,17 @@ def test_launch_count_follows_the_plan():
     class A:
         key_chunk = 0
         row_finish = 0
+        key_tile = 0
+        strip_slots = 0
         fp8 = False
 
     assert bench.kernel_launches_per_step(synth.shape("v4flash_s16k"), A) == 2
     assert bench.kernel_launches_per_step(synth.shape("tiny"), A) == 2
-    # top-2048 lists at S = 65,536 need three query blocks of the 512 MiB budget
+    # top-2048 lists at S = 65,536 need three query blocks of the 512 MiB
+    # budget, at S = 262,144 eleven
     assert bench.kernel_launches_per_step(synth.shape("large_s64k"), A) == 6
+    assert bench.kernel_launches_per_step(synth.shape("long_s256k"), A) == 22
+    assert bench.library_plan(synth.shape("long_s256k"), A)["query_blocks"] == 11
     A.fp8 = True
     assert bench.kernel_launches_per_step(synth.shape("v4flash_s16k"), A) == 4
     A.fp8 = False

@@ -90,3 +90,49 @@ def test_small_scratch_budget_many_blocks():
     oi, os_ = oracle.topk_scores(X, 2, 256)
     np.testing.assert_array_equal(gi.reshape(-1, 256).cpu().numpy(), oi)
     np.testing.assert_array_equal(gs.reshape(-1, 256).cpu().numpy().view(np.uint32), os_.view(np.uint32))
+
+
+# The fused kernel's own selection plans: the test entry selects with the
+# queries per tile, strip length, pool room and partial-list length the
+# indexer plans for that shape (si_options.plan_heads / plan_dim / plan_fp8),
+# so the pruning and radix-select steps the product runs are checked bit for
+# bit, not only through the end-to-end tolerance rule.
+PLANS = [
+    # H_I, d_I, fp8, k, S, T, m, key_chunk
+    (64, 128, 0, 512, 6000, 4096, 1, 0),     # V4-Flash step: 4 queries, 512-key strips
+    (64, 128, 0, 2048, 9000, 8192, 1, 0),    # top-2048 steps: half-width tile, 2 queries
+    (64, 128, 0, 512, 4000, 8192, 1, 1024),  # the sweep's chunked cells
+    (64, 128, 0, 1024, 4000, 8192, 1, 2048),
+    (8, 64, 0, 64, 2048, 512, 4, 0),         # tiny step: 32 queries, 128-key strips
+    (64, 128, 1, 512, 6000, 4096, 1, 0),     # FP8 plan of the V4-Flash step
+    (64, 128, 1, 2048, 9000, 8192, 1, 0),
+]
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "inf"])
+@pytest.mark.parametrize("H,D,fp8,k,S,T,m,chunk", PLANS)
+def test_bit_exact_on_the_indexer_plans(kind, H, D, fp8, k, S, T, m, chunk):
+    X = synth.gen_scores(1, S, T, seed=S + k + H, kind=kind)
+    opts = stl.options(key_chunk=chunk, plan_heads=H, plan_dim=D, plan_fp8=fp8)
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), m, k, opts=opts)
+    torch.cuda.synchronize()
+    assert stl.device_error() == 0
+    oi, os_ = oracle.topk_scores(X, m, k)
+    np.testing.assert_array_equal(gi.reshape(-1, k).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, k).cpu().numpy().view(np.uint32),
+                                  os_.view(np.uint32))
+
+
+@pytest.mark.parametrize("H,D,fp8,k", [(64, 128, 0, 512), (64, 128, 0, 2048)])
+def test_increasing_rows_on_the_indexer_plans(H, D, fp8, k):
+    """Scores rising along j on the product's plans: every key beats the
+    running k-th, every strip overflows the pools, every prune is exercised."""
+    S = T = 8192
+    X = np.broadcast_to(np.arange(T, dtype=np.float32), (1, S, T)).copy()
+    X += np.random.default_rng(1).standard_normal((1, S, T)).astype(np.float32) * 1e-3
+    opts = stl.options(plan_heads=H, plan_dim=D, plan_fp8=fp8)
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), 1, k, opts=opts)
+    oi, os_ = oracle.topk_scores(X, 1, k)
+    np.testing.assert_array_equal(gi.reshape(-1, k).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, k).cpu().numpy().view(np.uint32),
+                                  os_.view(np.uint32))

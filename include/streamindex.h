@@ -246,6 +246,20 @@ const char* si_status_string(int status);
  * the device error word of the current device. */
 int si_get_last_device_error(void* stream);
 
+/*
+ * si_role_cycles: per-CTA role counters of the profiling build of the library
+ * (compiled with SI_ROLE_CLOCKS): for each CTA of the fused score kernel, 32
+ * unsigned 64-bit words accumulated over every launch since the last reset --
+ * cycles each warp role spends in total, waiting on each of its barriers and
+ * in each selection phase, and event counts (units, key tiles, strips,
+ * appended keys, prunes, radix selects); the slot order is the RoleSlot enum
+ * of the library's device code.  Synchronises the device, copies the first
+ * n_words words ([CTA][32], at most 1024 CTAs) to host memory `out`, and
+ * zeroes them when `reset` is non-zero.  The normal build keeps no counters
+ * and returns SI_ERR_UNSUPPORTED.
+ */
+int si_role_cycles(uint64_t* out, int n_words, int reset);
+
 /* Library version as an integer, major*10000 + minor*100 + patch. */
 int si_version(void);
 

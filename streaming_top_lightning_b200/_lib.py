@@ -23,6 +23,7 @@ EXPORTS = [
     "si_indexer_topk", "si_indexer_topk_workspace_size", "si_indexer_topk_ex",
     "si_indexer_topk_fp8", "si_quantize_fp8_rows", "si_topk_scores", "si_status_string",
     "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc", "si_indexer_topk_plan",
+    "si_role_cycles",
 ]
 
 
@@ -57,11 +58,16 @@ class StreamIndexError(RuntimeError):
 _lib = None
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load the library (once) and declare argument types."""
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the library (once) and declare argument types.  The first call
+    fixes which build is used: the default one, or ``path`` (the profiling
+    build, libstreamindex_roles.so)."""
     global _lib
     if _lib is not None:
+        if path is not None and os.path.abspath(path) != os.path.abspath(_lib._name):
+            raise RuntimeError(f"{_lib._name} is already loaded")
         return _lib
+    path = path or LIB_PATH
     if not os.path.exists(path):
         raise ImportError(f"{path} is not built; run python -m streaming_top_lightning_b200.build")
     lib = ctypes.CDLL(path)
@@ -79,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.si_status_string.restype = ctypes.c_char_p
     lib.si_get_last_device_error.argtypes = [P]
     lib.si_version.argtypes = []
+    lib.si_role_cycles.argtypes = [P, I, I]
     for name in EXPORTS:
         if name != "si_status_string":
             getattr(lib, name).restype = I

@@ -20,6 +20,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libstreamindex.so")
+# profiling build: the same sources with per-role cycle counters (SI_ROLE_CLOCKS)
+LIB_ROLES = os.path.join(PKG, "libstreamindex_roles.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -35,32 +37,37 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
     deps += glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, debug: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into libstreamindex.so (skipped when up to date)."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, debug: bool = False, verbose: bool = False,
+          roles: bool = False) -> str:
+    """Compile every .cu under csrc/ into libstreamindex.so (skipped when up to
+    date); ``roles`` builds the profiling variant libstreamindex_roles.so."""
+    lib = LIB_ROLES if roles else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-lineinfo", "-O3", "-std=c++17", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC", "-shared", "--cudart", "static", "-I", INCLUDE, "-I", CSRC,
            "-o", tmp, *sources()]
     if debug:
         cmd.insert(1, "-DSI_DEBUG")
+    if roles:
+        cmd.insert(1, "-DSI_ROLE_CLOCKS")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, debug="--debug" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, debug="--debug" in sys.argv,
+                verbose="-v" in sys.argv, roles="--roles" in sys.argv))

@@ -22,6 +22,12 @@ namespace si {
 
 __device__ uint32_t g_err_word;
 
+#ifdef SI_ROLE_CLOCKS
+// role counters of the profiling build: [CTA][kRoleSlots]
+constexpr int kRoleCtas = 1024;
+__device__ unsigned long long g_role_cycles[kRoleCtas * kRoleSlots];
+#endif
+
 namespace {
 
 struct DevInfo {
@@ -30,6 +36,7 @@ struct DevInfo {
   int sms = 0;
   int max_smem = 0;
   uint32_t* err = nullptr;
+  unsigned long long* role = nullptr;  // profiling build: role counters
 };
 
 std::mutex g_mu;
@@ -52,6 +59,11 @@ int dev_info(DevInfo** out) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return SI_ERR_CUDA;
     d.err = static_cast<uint32_t*>(p);
+#ifdef SI_ROLE_CLOCKS
+    void* r = nullptr;
+    if (cudaGetSymbolAddress(&r, g_role_cycles) != cudaSuccess) return SI_ERR_CUDA;
+    d.role = static_cast<unsigned long long*>(r);
+#endif
     d.ok = (major == 10 && minor == 0);
     d.init = true;
   }
@@ -288,6 +300,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     p.nst = sp_plan.nst;
     p.nslot = sp_plan.nslot;
     p.debug_flags = o.debug_flags;
+    p.role = dev->role;
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -545,6 +558,25 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     rc = SI_ERR_CUDA;
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SI_OK) rc = SI_ERR_CUDA;
   return rc;
+}
+
+int si_role_cycles(uint64_t* out, int n_words, int reset) {
+#ifdef SI_ROLE_CLOCKS
+  if (!out && n_words > 0) return SI_ERR_NULL;
+  if (n_words < 0) return SI_ERR_DIM;
+  DevInfo* dev;
+  int rc = dev_info(&dev);
+  if (rc) return rc;
+  const size_t n = std::min((size_t)n_words, (size_t)kRoleCtas * kRoleSlots);
+  if (cudaDeviceSynchronize() != cudaSuccess) return SI_ERR_CUDA;
+  if (n && cudaMemcpyFromSymbol(out, g_role_cycles, n * sizeof(uint64_t)) != cudaSuccess)
+    return SI_ERR_CUDA;
+  if (reset && cudaMemset(dev->role, 0, sizeof(g_role_cycles)) != cudaSuccess) return SI_ERR_CUDA;
+  return SI_OK;
+#else
+  (void)out, (void)n_words, (void)reset;
+  return SI_ERR_UNSUPPORTED;
+#endif
 }
 
 int si_get_last_device_error(void* stream) {

@@ -185,11 +185,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = cs->tmem_base;
-  Ctl ctl{p.err, &cs->abort, p.timeout_ns};
+  Ctl ctl{p.err, &cs->abort, p.timeout_ns, p.role};
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
+      const long long t_role = role_t0();
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_kc);
       const uint64_t pol_q = policy_evict_first();
@@ -211,7 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int b = 0, g = 0, c = 0;
         const bool ok = unit_decode(p.ug, id, b, g, c);
         const int r = ring_it % kRing;
-        if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl)) return -1;
+        if (!mbar_wait(smem_u32(&cs->unit_empty[r]), ((ring_it / kRing) & 1u) ^ 1u, ctl,
+                       R_PROD_WAIT_UNIT))
+          return -1;
         u = UnitInfo{0, 0, 0, 0, 0, 0, 0};
         if (ok) {
           const int vmax = tile_vmax(p.ug, g);
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (u.ntiles > 0) {
           // query tile: rows (b*S + g*QT)*H .. +NQ of q viewed as [B*S*H, D]
-          if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl)) break;
+          if (!mbar_wait(smem_u32(&cs->q_empty), (q_it & 1u) ^ 1u, ctl, R_PROD_WAIT_Q)) break;
           const uint32_t qb = smem_u32(&cs->q_full);
           mbar_arrive_expect_tx(qb, G::kQBytes);
           const int qrow = (u.b * sp.S + u.g * QT) * H;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bool stop = false;
           for (int i = 0; i < u.ntiles; ++i) {
             const int s = kstage % NST;
-            if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl)) {
+            if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl, R_PROD_WAIT_KC)) {
               stop = true;
               break;
             }
@@ -282,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // drain: wait (bounded, regardless of abort) for every copy this thread
       // issued to land before the CTA may exit
-      Ctl drain_ctl{p.err, nullptr, p.timeout_ns};
+      Ctl drain_ctl{p.err, nullptr, p.timeout_ns, nullptr};
       uint32_t dummy = 0;
       drain_ctl.abort = &dummy;
       for (uint32_t n = (kstage > (uint32_t)NST ? kstage - NST : 0); n < kstage; ++n) {
@@ -291,31 +294,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(smem_u32(&cs->full[s]), (n / NST) & 1u, drain_ctl);
       }
       if (q_issued) mbar_wait(smem_u32(&cs->q_full), (q_it - 1) & 1u, drain_ctl);
+      role_add(ctl, R_PROD_TOTAL, t_role);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      const long long t_role = role_t0();
       constexpr uint32_t idesc = FP8 ? idesc_make(0, 0, kM, NQ) : idesc_make(1, 1, kM, NQ);
       uint32_t ring_it = 0, kstage = 0, acc_it = 0, q_it = 0;
       for (;;) {
         const int r = ring_it % kRing;
-        if (!mbar_wait(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl)) break;
+        if (!mbar_wait(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl, R_MMA_WAIT_UNIT))
+          break;
         const UnitInfo u = cs->ring[r];  // ordered after the acquiring wait
         mbar_arrive(smem_u32(&cs->unit_empty[r]));
         ++ring_it;
         if (!u.valid) break;
+        role_count(ctl, R_UNITS, 1);
+        role_count(ctl, R_TILES, (unsigned long long)u.ntiles);
         if (u.ntiles == 0) continue;
-        if (!mbar_wait(smem_u32(&cs->q_full), q_it & 1u, ctl)) break;
+        if (!mbar_wait(smem_u32(&cs->q_full), q_it & 1u, ctl, R_MMA_WAIT_Q)) break;
         tc_fence_after();
         bool stop = false;
         for (int i = 0; i < u.ntiles; ++i) {
           const int s = kstage % NST;
-          if (!mbar_wait(smem_u32(&cs->full[s]), (kstage / NST) & 1u, ctl)) {
+          if (!mbar_wait(smem_u32(&cs->full[s]), (kstage / NST) & 1u, ctl, R_MMA_WAIT_KC)) {
             stop = true;
             break;
           }
           const int ab = acc_it & 1;
-          if (!mbar_wait(smem_u32(&cs->acc_empty[ab]), ((acc_it >> 1) & 1u) ^ 1u, ctl)) {
+          if (!mbar_wait(smem_u32(&cs->acc_empty[ab]), ((acc_it >> 1) & 1u) ^ 1u, ctl,
+                         R_MMA_WAIT_ACC)) {
             stop = true;
             break;
           }
@@ -343,8 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: all MMAs issued by this thread complete before TMEM is freed
       umma_commit(smem_u32(&cs->drain));
       uint32_t dummy = 0;
-      Ctl drain_ctl{p.err, &dummy, p.timeout_ns};
+      Ctl drain_ctl{p.err, &dummy, p.timeout_ns, nullptr};
       mbar_wait(smem_u32(&cs->drain), 0u, drain_ctl);
+      role_add(ctl, R_MMA_TOTAL, t_role);
     }
   } else if (warp < kSelWarp0) {
     // ---------------------------------------------------------- epilogue
@@ -357,9 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kl = quad * 32 + lane;  // key within the tile
     float* wq = w_s + ew * kHalfN;    // this warp's private copy of its half's weights
     uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
+    const long long t_role = role_t0();
     for (;;) {
       const int r = ring_it % kRing;
-      if (!mbar_wait_warp(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl)) break;
+      if (!mbar_wait_warp(smem_u32(&cs->unit_full[r]), (ring_it / kRing) & 1u, ctl,
+                          R_EPI_WAIT_UNIT))
+        break;
       const UnitInfo u = cs->ring[r];  // ordered after the acquiring wait
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&cs->unit_empty[r]));
@@ -406,14 +419,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = (int)(strip_it % (uint32_t)NSL);
         if (pos == 0) {
           if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u,
-                              ctl)) {
+                              ctl, R_EPI_WAIT_STRIP)) {
             stop = true;
             break;
           }
         }
         if (u.ntiles > 0) {
           const int ab = acc_it & 1;
-          if (!mbar_wait_warp(smem_u32(&cs->acc_full[ab]), (acc_it >> 1) & 1u, ctl)) {
+          if (!mbar_wait_warp(smem_u32(&cs->acc_full[ab]), (acc_it >> 1) & 1u, ctl, R_EPI_WAIT_ACC)) {
             stop = true;
             break;
           }
@@ -485,6 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (stop) break;
     }
+    if (lane == 0) role_add(ctl, R_EPI_TOTAL, t_role);
   } else {
     // ---------------------------------------------------------- selection
     sm.strip = strip;

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   }
   __syncthreads();
 
-  Ctl ctl{err, &misc->abort, timeout_ns};
+  Ctl ctl{err, &misc->abort, timeout_ns, nullptr};
   sm.strip = strip;
   sm.meta = meta;
   sm.full_bar = full_bar;

@@ -50,11 +50,48 @@ SI_DEV float key_score(uint64_t k) {
 SI_DEV int key_index(uint64_t k) { return 0x7FFFFFFF - (int)((uint32_t)k >> 1); }
 
 // ------------------------------------------------------------------ control
+// Per-CTA role counters of a profiling build (compiled with SI_ROLE_CLOCKS):
+// cycles each role spends in total, waiting on each barrier and in each
+// selection phase, and event counts.  They cost nothing in the normal build.
+enum RoleSlot {
+  R_PROD_TOTAL = 0, R_PROD_WAIT_KC, R_PROD_WAIT_Q, R_PROD_WAIT_UNIT,
+  R_MMA_TOTAL, R_MMA_WAIT_KC, R_MMA_WAIT_ACC, R_MMA_WAIT_Q, R_MMA_WAIT_UNIT,
+  R_EPI_TOTAL, R_EPI_WAIT_UNIT, R_EPI_WAIT_STRIP, R_EPI_WAIT_ACC,
+  R_SEL_TOTAL, R_SEL_WAIT_STRIP, R_SEL_INTAKE, R_SEL_UNIT_END, R_SEL_PRUNE_CYC,
+  R_SEL_PRUNES, R_SEL_SHRINKS, R_SEL_APPENDS, R_SEL_STRIPS, R_SEL_END_WAIT,
+  R_UNITS, R_TILES, R_SEL_KEYS, kRoleSlots = 32
+};
+
 struct Ctl {
   uint32_t* err;             // global error word
   volatile uint32_t* abort;  // CTA-wide abort flag in shared memory
   uint64_t timeout_ns;       // limit for any single wait
+  unsigned long long* role;  // [grid][kRoleSlots] counters (profiling build), else null
 };
+
+SI_DEV long long role_t0() {
+#ifdef SI_ROLE_CLOCKS
+  return clock64();
+#else
+  return 0;
+#endif
+}
+// Add the cycles since t0 to a role counter (lane 0 of a warp, or a single thread).
+SI_DEV void role_add(const Ctl& c, int slot, long long t0) {
+#ifdef SI_ROLE_CLOCKS
+  if (slot >= 0 && c.role)
+    atomicAdd(&c.role[blockIdx.x * kRoleSlots + slot], (unsigned long long)(clock64() - t0));
+#else
+  (void)c, (void)slot, (void)t0;
+#endif
+}
+SI_DEV void role_count(const Ctl& c, int slot, unsigned long long v) {
+#ifdef SI_ROLE_CLOCKS
+  if (c.role) atomicAdd(&c.role[blockIdx.x * kRoleSlots + slot], v);
+#else
+  (void)c, (void)slot, (void)v;
+#endif
+}
 
 SI_DEV uint64_t globaltimer() {
   uint64_t t;
@@ -98,7 +135,20 @@ SI_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Returns false if the
 // CTA is aborting or the wait exceeded the time limit (then it raises abort).
-SI_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+// A profiling build adds the wait's cycles to role counter `slot` (if >= 0).
+SI_DEV bool mbar_wait_(uint32_t bar, uint32_t parity, const Ctl& c);
+SI_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c, int slot = -1) {
+#ifdef SI_ROLE_CLOCKS
+  const long long t = role_t0();
+  const bool r = mbar_wait_(bar, parity, c);
+  role_add(c, slot, t);
+  return r;
+#else
+  (void)slot;
+  return mbar_wait_(bar, parity, c);
+#endif
+}
+SI_DEV bool mbar_wait_(uint32_t bar, uint32_t parity, const Ctl& c) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t n = 0;
@@ -117,7 +167,19 @@ SI_DEV bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
 // Warp-collective form: every lane returns the same answer, so the warp can
 // go on to warp-synchronous code (shuffles, __syncwarp) without diverging.
 // Each lane performs its own acquiring try_wait before it returns true.
-SI_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, const Ctl& c) {
+SI_DEV bool mbar_wait_warp_(uint32_t bar, uint32_t parity, const Ctl& c);
+SI_DEV bool mbar_wait_warp(uint32_t bar, uint32_t parity, const Ctl& c, int slot = -1) {
+#ifdef SI_ROLE_CLOCKS
+  const long long t = role_t0();
+  const bool r = mbar_wait_warp_(bar, parity, c);
+  if ((threadIdx.x & 31u) == 0u) role_add(c, slot, t);
+  return r;
+#else
+  (void)slot;
+  return mbar_wait_warp_(bar, parity, c);
+#endif
+}
+SI_DEV bool mbar_wait_warp_(uint32_t bar, uint32_t parity, const Ctl& c) {
   const uint32_t lane = threadIdx.x & 31u;
   uint64_t t0 = 0;
   for (uint32_t n = 0;; ++n) {

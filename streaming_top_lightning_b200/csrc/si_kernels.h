@@ -22,6 +22,7 @@ struct ScoreParams {
   int nst;             // key-tile pipeline stages
   int nslot;           // strip ring slots
   int debug_flags;     // bit 0: skip the first key-tile load (timeout test)
+  unsigned long long* role;  // role counters of a profiling build, else null
 };
 
 // Shared-memory plan of the fused kernel for one problem shape.

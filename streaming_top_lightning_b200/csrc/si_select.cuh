@@ -282,10 +282,12 @@ static __device__ __noinline__ bool pool_prune(uint64_t* pool, int* np_io, int K
 // step, the steps that fit are stored, the pool is pruned and the rest of the
 // chunk is compared again with the new threshold.
 SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t* pool, int cap,
-                            int K, int* np_p, uint64_t* th_p, uint32_t* hist, int lane) {
+                            int K, int* np_p, uint64_t* th_p, uint32_t* hist, int lane,
+                            const Ctl& ctl) {
   int lim = V - j0;
   if (lim > nkeys) lim = nkeys;
   if (lim <= 0) return;
+  if (lane == 0) role_count(ctl, R_SEL_KEYS, (unsigned long long)lim);
   uint64_t theta = *th_p;
   int np = *np_p;
   // theta 0 takes every key (-inf >= -inf too)
@@ -334,15 +336,20 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
         }
       }
       np += add;
+      if (lane == 0) role_count(ctl, R_SEL_APPENDS, (unsigned long long)add);
       s0 = s1;
       if (s0 < nsteps) {
         // the pool cannot take step s0: raise theta, then compare the rest again
+        const long long t_p = role_t0();
         __syncwarp();
+        if (lane == 0) role_count(ctl, R_SEL_PRUNES, 1);
         if (!pool_prune(pool, &np, K, &theta, lane) || np + 64 > cap) {
+          if (lane == 0) role_count(ctl, R_SEL_SHRINKS, 1);
           theta = pool_shrink(pool, np, K, hist, lane);
           np = K;
         }
         thf = key_score(theta);
+        if (lane == 0) role_add(ctl, R_SEL_PRUNE_CYC, t_p);
       }
     }
   }
@@ -496,20 +503,25 @@ __host__ __device__ constexpr bool rows_sorted_in_warp(int K) { return K <= 512;
 // query's keys) or leaves a pruned partial list for the merge kernel.
 SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, int sw, int lane) {
   uint32_t* hist = sm.hist + sw * 256;
+  const long long t_role = role_t0();
   for (uint32_t it = 0;; ++it) {
     const int slot = (int)(it % (uint32_t)sm.nslot);
     const uint32_t ph = (it / (uint32_t)sm.nslot) & 1u;
-    if (!mbar_wait_warp(sm.full_bar + 8 * slot, ph, ctl)) return;
+    if (!mbar_wait_warp(sm.full_bar + 8 * slot, ph, ctl, R_SEL_WAIT_STRIP)) break;
     const StripMeta md = sm.meta[slot];  // ordered after the acquiring wait
-    if (!md.valid) return;
+    if (!md.valid) break;
+    if (lane == 0) role_count(ctl, R_SEL_STRIPS, 1);
     const float* st = sm.strip + (size_t)slot * p.QT * p.CS;
     for (int qi = sw; qi < p.QT; qi += kSelWarps) {
       const int t = md.g * p.QT + qi;
       if (t >= p.S) continue;
       uint64_t* pool = sm.pool + (size_t)qi * p.cap;
+      const long long t_in = role_t0();
       pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), pool,
-                      p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane);
+                      p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane, ctl);
+      if (lane == 0) role_add(ctl, R_SEL_INTAKE, t_in);
       if (md.last) {
+        const long long t_end = role_t0();
         if (p.final_rows) {
           const int64_t o = ((int64_t)md.b * p.S + t) * p.K;
           finish_row(pool, sm.npool[qi], p.K, hist, p.out_idx + o, p.out_score + o, lane);
@@ -520,6 +532,7 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
         if (lane == 0) {
           sm.npool[qi] = 0;
           sm.theta[qi] = 0ull;
+          role_add(ctl, R_SEL_UNIT_END, t_end);
         }
         __syncwarp();
       }
@@ -527,6 +540,7 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
     __syncwarp();
     mbar_arrive(sm.empty_bar + 8 * slot);
   }
+  if (lane == 0) role_add(ctl, R_SEL_TOTAL, t_role);
 }
 
 // Shared-memory bytes of the selection state for QT queries (pools,

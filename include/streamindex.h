@@ -33,9 +33,8 @@
  *    d_I in {64, 128}; 1 <= topk <= 2048; B*S*H_I < 2^31; pointers 16-byte
  *    aligned.  The selection keeps a candidate pool per query of a query
  *    tile in shared memory, so with few heads (many queries per tile) the
- *    largest topk is lower: bf16 H_I=8: 768 (d_I=128), 1152 (d_I=64);
- *    bf16 H_I=16, d_I=128: 1728; FP8 H_I=8: 1152 (d_I=128), 1344 (d_I=64);
- *    2048 otherwise.  A larger topk returns SI_ERR_TOPK.
+ *    largest topk is lower: bf16 H_I=8: 1056 (d_I=128), 1312 (d_I=64);
+ *    FP8 H_I=8: 1280 (d_I=128), 1408 (d_I=64); 2048 otherwise.  A larger topk returns SI_ERR_TOPK.
  */
 #ifndef STREAMINDEX_H
 #define STREAMINDEX_H

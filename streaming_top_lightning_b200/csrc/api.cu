@@ -163,11 +163,12 @@ int read_opts(const si_options* o, Opts* out) {
 // rows themselves: no partial lists, one launch block, no merge.
 struct Plan {
   int QT, G, T, C, nch_max, L, tb, n_blocks, final_rows;
-  size_t counters_bytes, partial_bytes;
-  size_t ws_bytes() const { return align256(counters_bytes) + partial_bytes; }
+  size_t counters_bytes, tail_bytes, partial_bytes;
+  // unit counter | padded copy of the last query tile's weights | partial lists
+  size_t ws_bytes() const { return align256(counters_bytes) + align256(tail_bytes) + partial_bytes; }
 };
 
-Plan make_plan(int B, int S, int T, int K, int QT, const Opts& o) {
+Plan make_plan(int B, int S, int T, int K, int QT, int H, const Opts& o) {
   Plan p{};
   p.QT = QT;
   p.T = T;
@@ -196,6 +197,7 @@ Plan make_plan(int B, int S, int T, int K, int QT, const Opts& o) {
     p.n_blocks = (p.G + p.tb - 1) / p.tb;
   }
   p.counters_bytes = sizeof(int);  // one unit counter shared by every launch
+  p.tail_bytes = (size_t)QT * H * sizeof(float);  // one query tile's weights (0: none)
   return p;
 }
 
@@ -210,6 +212,16 @@ cudaError_t finish_launch(const uint64_t* partial, const SelParams& sp, const Un
 // True when no row-sort pass is needed after the finishing launches.
 bool rows_come_sorted(const Plan& pl, int K) {
   return rows_sorted_in_warp(K) || (!pl.final_rows && pl.nch_max == 1);
+}
+
+// The selection's invariant: a pool has room for K keys plus one 64-key
+// step (appends are checked step by step, and a prune or an exact select
+// leaves at most cap - 64 keys), strips are whole warps of keys, and a partial
+// list holds at least K keys.  Checked before every launch that runs the
+// streaming selection.
+bool sel_params_ok(const SelParams& sp) {
+  return sp.cap >= ((sp.K + 64 + 31) / 32) * 32 && sp.CS >= 32 && sp.CS % 32 == 0 &&
+         sp.L >= sp.K;
 }
 
 // Kernel launches of one call: a score launch per query block, a finishing
@@ -255,14 +267,25 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   if ((rc = dev_info(&dev))) return rc;
   const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile, o.strip_slots);
   if ((rc = plan_status(sp_plan))) return rc;  // pools of this topk do not fit, or key_tile
-  const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, o);
+  const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, H, o);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
   if (!aligned16(ws)) return SI_ERR_ALIGN;
 
   int* counters = static_cast<int*>(ws);
-  uint64_t* partial =
-      reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + align256(pl.counters_bytes));
+  float* w_tail = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(pl.counters_bytes));
+  uint64_t* partial = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(w_tail) +
+                                                  align256(pl.tail_bytes));
   if (cudaMemsetAsync(counters, 0, pl.counters_bytes, stream) != cudaSuccess) return SI_ERR_CUDA;
+  // the last batch's last query tile, when S is not a multiple of its
+  // queries, gets a zero-padded copy of its rows of w to read (bf16 path)
+  if (!fp8 && S % pl.QT != 0) {
+    const int valid = S % pl.QT;
+    const int64_t row0 = (int64_t)(B - 1) * S + (int64_t)(pl.G - 1) * pl.QT;
+    if (cudaMemsetAsync(w_tail, 0, (size_t)pl.QT * H * sizeof(float), stream) != cudaSuccess ||
+        cudaMemcpyAsync(w_tail, w + row0 * H, (size_t)valid * H * sizeof(float),
+                        cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+      return SI_ERR_CUDA;
+  }
 
   const int esz = fp8 ? 1 : 2;
   const int row_bytes = D * esz;
@@ -292,6 +315,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
                       out_idx, out_score, partial, pl.final_rows};
     p.ug = ug;
     p.w = w;
+    p.w_tail = w_tail;
     p.s_q = s_q;
     p.s_k = s_k;
     p.counter = counters;
@@ -301,6 +325,7 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     p.nslot = sp_plan.nslot;
     p.debug_flags = o.debug_flags;
     p.role = dev->role;
+    if (!sel_params_ok(p.sel)) return SI_ERR_TOPK;
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -309,7 +334,8 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
       return SI_ERR_CUDA;
     const bool blk_ev = o.ev_list && 2 * blk + 1 < o.ev_count;
     if (blk_ev && cudaEventRecord(o.ev_list[2 * blk], stream) != cudaSuccess) return SI_ERR_CUDA;
-    if (launch_score_topk(fp8, D, H, sp_plan.nq, tm_q, tm_kc, p, grid, sp_plan.smem, stream) !=
+    if (launch_score_topk(fp8, D, H, sp_plan.nq, tm_q, tm_kc, p, grid, sp_plan.smem,
+                          stream) !=
         cudaSuccess)
       return SI_ERR_CUDA;
     if (blk_ev && cudaEventRecord(o.ev_list[2 * blk + 1], stream) != cudaSuccess)
@@ -335,8 +361,8 @@ int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_o
   Opts o;
   if ((rc = read_opts(opt, &o))) return rc;
   // the larger need of the two query-tile widths the score plan may choose
-  const Plan full = make_plan(B, S, S / m, K, 256 / H, o);
-  const Plan half = make_plan(B, S, S / m, K, 128 / H, o);
+  const Plan full = make_plan(B, S, S / m, K, 256 / H, H, o);
+  const Plan half = make_plan(B, S, S / m, K, 128 / H, H, o);
   *bytes = std::max(full.ws_bytes(), half.ws_bytes());
   (void)fp8;
   return SI_OK;
@@ -434,7 +460,7 @@ int si_indexer_topk_plan(int B, int S, int H_I, int d_I, int m, int topk, int fp
   plan_limits(&max_smem, &sms);
   const ScorePlan sp = plan_score(fp8 != 0, d_I, H_I, topk, max_smem, o.key_tile, o.strip_slots);
   if ((rc = plan_status(sp))) return rc;
-  const Plan pl = make_plan(B, S, S / m, topk, sp.QT, o);
+  const Plan pl = make_plan(B, S, S / m, topk, sp.QT, H_I, o);
   si_plan_info r{};
   r.queries_per_tile = sp.QT;
   r.mma_n = sp.nq;
@@ -522,10 +548,10 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     QT = fp.QT;
     CS = fp.CS;
     cap = fp.cap;
-    if (topk_scores_smem_bytes(QT, cap, CS) > (size_t)dev->max_smem) return SI_ERR_TOPK;
   }
+  if (topk_scores_smem_bytes(QT, cap, CS) > (size_t)dev->max_smem) return SI_ERR_TOPK;
   // the selection-only path sees T keys per row; m still sets visibility
-  const Plan pl = make_plan(B, S, T, topk, QT, o);
+  const Plan pl = make_plan(B, S, T, topk, QT, 0, o);
   const size_t bytes = pl.ws_bytes();
   void* ws = nullptr;
   if (cudaMallocAsync(&ws, bytes, st) != cudaSuccess) return SI_ERR_CUDA;
@@ -546,6 +572,10 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
     if (grid < 1) grid = 1;
+    if (!sel_params_ok(sp)) {
+      rc = SI_ERR_TOPK;
+      break;
+    }
     if (launch_topk_scores(scores, sp, ug, counters, dev->err,
                            (uint64_t)o.timeout_ms * 1000000ull, grid, st) != cudaSuccess)
       rc = SI_ERR_CUDA;

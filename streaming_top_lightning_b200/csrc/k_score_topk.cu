@@ -41,7 +41,6 @@ constexpr int kM = 128;         // MMA M: keys per tile
 constexpr int kEpiWarp0 = 2;    // first epilogue warp
 constexpr int kEpiWarps = 8;    // two per TMEM lane quadrant, one per column half
 constexpr int kEpiThreads = kEpiWarps * 32;
-constexpr int kHalfN = kN / 2;  // largest accumulator column count per epilogue warp
 constexpr int kSelWarp0 = kEpiWarp0 + kEpiWarps;  // first selection warp
 constexpr int kMaxSlots = 4;    // score-strip ring slots at most
 static_assert(kThreads == (kSelWarp0 + kSelWarps) * 32, "warp roles");
@@ -72,6 +71,8 @@ struct OperandGeom {
   static constexpr int kKSteps = kRowBytes / 32;                  // MMA instructions per tile
   static constexpr int kQBytes = NQ * kRowBytes;
   static constexpr int kKcBytes = kM * kRowBytes;
+  static constexpr int kKbBytes = kM * kSw;       // one K-block of a key tile: a ring slot
+  static constexpr int kPerBlock = kSw / 32;      // MMA instructions per K-block
 };
 
 template <int SW>
@@ -94,29 +95,32 @@ SI_DEV void tmem_ld_fence(float (&v)[32]) {
 }
 
 // Independent packed accumulators per query of an epilogue warp: enough
-// chains to cover the FMA latency, at most 8 float2 in all.  HALF is the
-// warp's column count (half of the MMA N).
-template <int H, int HALF>
+// chains to cover the FMA latency, at most 8 float2 in all.  COLS is the
+// warp's column count (its share of the MMA N).
+template <int H, int COLS>
 struct EpiGeom {
-  static constexpr int kQH = HALF / H;                 // queries per column half
+  static constexpr int kQH = COLS / H;                 // queries of the warp's columns
   static constexpr int kNA = kQH >= 8 ? 1 : 8 / kQH;   // chains per query
-  static_assert(kQH * kNA <= 16 && (H / 2) % kNA == 0, "accumulator split");
+  static_assert(kQH * kNA <= 32 && (H / 2) % kNA == 0, "accumulator split");
 };
 
-// Weighted ReLU head sum of one 32-column chunk of this warp's column half
-// into the packed accumulators.  Local column c = ch*32 + e is query c / H of
-// the half and head c % H; head pair (c % H)/2 feeds chain ((c % H)/2) % kNA.
-// w4 holds the half's weights as float4 groups (one LDS.128 per 4 columns).
-template <int H, int HALF>
-SI_DEV void epi_chunk(int ch, const float (&v)[32], const float4* w4,
-                      float2 (&acc)[EpiGeom<H, HALF>::kQH][EpiGeom<H, HALF>::kNA]) {
-  constexpr int NA = EpiGeom<H, HALF>::kNA;
+// Weighted ReLU head sum of one 32-column chunk of this warp's columns into
+// the packed accumulators.  Local column c = ch*32 + e is query c / H of the
+// warp and head c % H; head pair (c % H)/2 feeds chain ((c % H)/2) % kNA.
+// wsrc: the warp's weights, contiguous -- global memory for bf16 (read as
+// float4 through the read-only path; the same 16 bytes in every lane, one L1
+// wavefront), the shared-memory copy for FP8.
+template <bool FP8, int H, int COLS>
+SI_DEV void epi_chunk(int ch, const float (&v)[32], const float* wsrc,
+                      float2 (&acc)[EpiGeom<H, COLS>::kQH][EpiGeom<H, COLS>::kNA]) {
+  constexpr int NA = EpiGeom<H, COLS>::kNA;
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     const int col = ch * 32 + e;
     const int ql = col / H;
     const int a0 = ((col % H) >> 1) % NA, a1 = (((col + 2) % H) >> 1) % NA;
-    const float4 wv = w4[col >> 2];
+    const float4 wv = FP8 ? *reinterpret_cast<const float4*>(wsrc + col)
+                          : __ldg(reinterpret_cast<const float4*>(wsrc + col));
     const float2 r0 = make_float2(fmaxf(v[e], 0.0f), fmaxf(v[e + 1], 0.0f));
     const float2 r1 = make_float2(fmaxf(v[e + 2], 0.0f), fmaxf(v[e + 3], 0.0f));
     acc[ql][a0] = __ffma2_rn(make_float2(wv.x, wv.y), r0, acc[ql][a0]);
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  const ScoreParams p) {
   using G = OperandGeom<FP8, D, NQ>;
   constexpr int QT = NQ / H;
-  constexpr int HALF = NQ / 2;  // accumulator columns per epilogue warp
+  constexpr int COLS = NQ / 2;  // accumulator columns per epilogue warp (a column half)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -141,13 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint8_t* q_s = smem;
   uint8_t* kc_s = q_s + G::kQBytes;
-  float* strip = reinterpret_cast<float*>(kc_s + (size_t)NST * G::kKcBytes);
+  float* strip = reinterpret_cast<float*>(kc_s + (size_t)NST * G::kKbBytes);
   uint8_t* sel_base = reinterpret_cast<uint8_t*>(strip + (size_t)NSL * QT * CS);
   SelSmem sm;
   sel_state_carve(sel_base, QT, sp.cap, sm);
-  // [kEpiWarps][kHalfN]: each epilogue warp's private copy of its half of the weights
+  // FP8 only, [kEpiWarps][COLS]: each epilogue warp's copy of its columns'
+  // weights folded with the query row scales
   float* w_s = reinterpret_cast<float*>(sel_base + sel_state_bytes(QT, sp.cap));
-  ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + kEpiWarps * kHalfN);
+  ScoreCtlSmem* cs = reinterpret_cast<ScoreCtlSmem*>(w_s + (FP8 ? kEpiWarps * COLS : 0));
 
   const uint32_t q_addr = smem_u32(q_s), kc_addr = smem_u32(kc_s);
   if (tid == 0) {
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < NSL; ++i) {
       mbar_init(smem_u32(&cs->strip_full[i]), kEpiThreads);
-      mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);
+      mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);  // every selection lane
     }
     mbar_init(smem_u32(&cs->q_full), 1);
     mbar_init(smem_u32(&cs->q_empty), 1);
@@ -255,28 +260,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pol_q);
           q_issued = true;
           ++q_it;
-          // key tiles
+          // key tiles, one K-block (kM keys x kSw bytes) per ring slot
           bool stop = false;
-          for (int i = 0; i < u.ntiles; ++i) {
-            const int s = kstage % NST;
-            if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl, R_PROD_WAIT_KC)) {
-              stop = true;
-              break;
-            }
-            const uint32_t fb = smem_u32(&cs->full[s]);
-            mbar_arrive_expect_tx(fb, G::kKcBytes);
-            if ((p.debug_flags & 1) && !skipped) {
-              skipped = true;  // the consumer's wait on this stage must expire
-              skipped_stage = s;
-            } else {
-              const int krow = u.b * sp.T + u.kbeg + i * kM;
-              const uint32_t dst = kc_addr + s * G::kKcBytes;
-#pragma unroll
-              for (int kb = 0; kb < G::kKBlocks; ++kb)
-                tma_load_2d(dst + kb * (kM * G::kSw), &tm_kc, fb, kb * (G::kSw / G::kEsz), krow,
+          for (int i = 0; i < u.ntiles && !stop; ++i) {
+            const int krow = u.b * sp.T + u.kbeg + i * kM;
+            for (int kb = 0; kb < G::kKBlocks; ++kb) {
+              const int s = kstage % NST;
+              if (!mbar_wait(smem_u32(&cs->empty[s]), ((kstage / NST) & 1u) ^ 1u, ctl,
+                             R_PROD_WAIT_KC)) {
+                stop = true;
+                break;
+              }
+              const uint32_t fb = smem_u32(&cs->full[s]);
+              mbar_arrive_expect_tx(fb, G::kKbBytes);
+              if ((p.debug_flags & 1) && !skipped) {
+                skipped = true;  // the consumer's wait on this slot must expire
+                skipped_stage = s;
+              } else {
+                tma_load_2d(kc_addr + s * G::kKbBytes, &tm_kc, fb, kb * (G::kSw / G::kEsz), krow,
                             pol_k);
+              }
+              ++kstage;
             }
-            ++kstage;
           }
           if (stop) break;
         }
@@ -316,33 +321,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(smem_u32(&cs->q_full), q_it & 1u, ctl, R_MMA_WAIT_Q)) break;
         tc_fence_after();
         bool stop = false;
-        for (int i = 0; i < u.ntiles; ++i) {
-          const int s = kstage % NST;
-          if (!mbar_wait(smem_u32(&cs->full[s]), (kstage / NST) & 1u, ctl, R_MMA_WAIT_KC)) {
-            stop = true;
-            break;
-          }
+        for (int i = 0; i < u.ntiles && !stop; ++i) {
           const int ab = acc_it & 1;
           if (!mbar_wait(smem_u32(&cs->acc_empty[ab]), ((acc_it >> 1) & 1u) ^ 1u, ctl,
                          R_MMA_WAIT_ACC)) {
             stop = true;
             break;
           }
-          tc_fence_after();
           const uint32_t d_tmem = tmem + ab * NQ;
-          const uint32_t a0 = kc_addr + s * G::kKcBytes;
+          // the tile's K-blocks, one ring slot each; a slot is released as
+          // soon as its MMAs have read it
 #pragma unroll
-          for (int k = 0; k < G::kKSteps; ++k) {
-            constexpr int kPerBlock = G::kSw / 32;
-            const int kb = k / kPerBlock, kin = k % kPerBlock;
-            const uint64_t ad = sdesc<G::kSw>(a0 + kb * (kM * G::kSw) + kin * 32);
-            const uint64_t bd = sdesc<G::kSw>(q_addr + kb * (NQ * G::kSw) + kin * 32);
-            if (FP8) umma_f8(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
-            else umma_bf16(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+          for (int kb = 0; kb < G::kKBlocks; ++kb) {
+            const int s = kstage % NST;
+            if (!mbar_wait(smem_u32(&cs->full[s]), (kstage / NST) & 1u, ctl, R_MMA_WAIT_KC)) {
+              stop = true;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = kc_addr + s * G::kKbBytes;
+#pragma unroll
+            for (int kin = 0; kin < G::kPerBlock; ++kin) {
+              const uint64_t ad = sdesc<G::kSw>(a0 + kin * 32);
+              const uint64_t bd = sdesc<G::kSw>(q_addr + kb * (NQ * G::kSw) + kin * 32);
+              const uint32_t acc = (kb > 0 || kin > 0) ? 1u : 0u;
+              if (FP8) umma_f8(d_tmem, ad, bd, idesc, acc);
+              else umma_bf16(d_tmem, ad, bd, idesc, acc);
+            }
+            umma_commit(smem_u32(&cs->empty[s]));
+            ++kstage;
           }
-          umma_commit(smem_u32(&cs->empty[s]));
+          if (stop) break;
           umma_commit(smem_u32(&cs->acc_full[ab]));
-          ++kstage;
           ++acc_it;
         }
         if (stop) break;
@@ -358,14 +368,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kSelWarp0) {
     // ---------------------------------------------------------- epilogue
-    using EG = EpiGeom<H, HALF>;
-    constexpr int QH = EG::kQH, NA = EG::kNA;
-    static_assert(HALF == 128 || HALF == 64, "epilogue chunk schedule");
-    const int ew = warp - kEpiWarp0;  // 0..7
+    using EG = EpiGeom<H, COLS>;
+    constexpr int QH = EG::kQH, NA = EG::kNA, NCH = COLS / 32;
+    static_assert(NCH % 2 == 0, "epilogue chunk schedule");
+    const int ew = warp - kEpiWarp0;  // 0 .. kEpiWarps-1
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;         // column half: queries [half*QH, half*QH + QH)
+    const int cb = ew >> 2;           // column block: queries [cb*QH, cb*QH + QH)
     const int kl = quad * 32 + lane;  // key within the tile
-    float* wq = w_s + ew * kHalfN;    // this warp's private copy of its half's weights
     uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
     const long long t_role = role_t0();
     for (;;) {
@@ -387,29 +396,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       // the unit's weights.  bf16: read in place from global memory (the
-      // warp's 128 columns are contiguous in w); every lane reads the same
-      // 16 bytes, which costs the L1 one wavefront where a shared-memory
-      // broadcast of 16 bytes costs four, and these reads would otherwise
-      // fill the shared-memory pipe.  FP8 (weights folded with the query row
-      // scales, which are positive, so relu(s*x) = s*relu(x)) and the last,
-      // partial tile of the last batch (whose rows past S lie outside w) take
-      // a zero-padded copy in shared memory.
+      // warp's columns are contiguous in w); every lane reads the same 16
+      // bytes, which costs the L1 one wavefront where a shared-memory
+      // broadcast of 16 bytes costs four.  Rows past S of a last, partial
+      // tile are the next batch's rows, whose scores are never used, except
+      // in the last batch, whose tile reads the zero-padded copy the host
+      // made in the workspace instead of reading past the end of w.  FP8: a
+      // copy in shared memory of the weights folded with the query row
+      // scales (positive, so relu(s*x) = s*relu(x)), zero past S.
       const int64_t wrow = (int64_t)u.b * sp.S + (int64_t)u.g * QT;
-      const bool w_direct = !FP8 && !(u.b == sp.B - 1 && (u.g + 1) * QT > sp.S);
-      const float4* w4 = reinterpret_cast<const float4*>(p.w + wrow * H + half * HALF);
-      if (!w_direct) {
-        for (int i = lane; i < HALF; i += 32) {
-          const int col = half * HALF + i;  // column of the query tile's N columns
+      const bool tail = u.b == sp.B - 1 && (u.g + 1) * QT > sp.S;
+      const float* wsrc = (tail ? p.w_tail : p.w + wrow * H) + cb * COLS;
+      if (FP8) {
+        float* wq = w_s + ew * COLS;
+        for (int i = lane; i < COLS; i += 32) {
+          const int col = cb * COLS + i;  // column of the query tile's N columns
           float wv = 0.0f;
-          if (u.g * QT + col / H < sp.S) {
-            wv = p.w[wrow * H + col];
-            if (FP8) wv *= p.s_q[wrow * H + col];
-          }
+          if (u.g * QT + col / H < sp.S) wv = p.w[wrow * H + col] * p.s_q[wrow * H + col];
           wq[i] = wv;
         }
-        w4 = reinterpret_cast<const float4*>(wq);
+        __syncwarp();
+        wsrc = wq;
       }
-      __syncwarp();
       int pos = 0, j_strip = u.kbeg;
       const int sp_chunk = p.ug.C;  // keys per chunk (a multiple of 128)
       int chunk_next = u.kbeg + sp_chunk;  // end of the current key chunk
@@ -431,40 +439,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t taddr =
-              tmem + ((uint32_t)(quad * 32) << 16) + ab * NQ + half * HALF;
+          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ab * NQ + cb * COLS;
           float2 acc[QH][NA];
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql)
 #pragma unroll
             for (int a = 0; a < NA; ++a) acc[ql][a] = make_float2(0.0f, 0.0f);
+          // 32 columns per TMEM load, two loads in flight: chunk c + 2 is read
+          // while chunk c is summed
           float va[32], vb[32];
           tmem_ld32(taddr, va);
           tmem_ld32(taddr + 32, vb);
           tmem_ld_wait();
           tmem_ld_fence(va);
           tmem_ld_fence(vb);
-          if constexpr (HALF == 128) {
-            epi_chunk<H, HALF>(0, va, w4, acc);
-            tmem_ld32(taddr + 64, va);
-            epi_chunk<H, HALF>(1, vb, w4, acc);
-            tmem_ld32(taddr + 96, vb);
-            tmem_ld_wait();
-            tmem_ld_fence(va);
-            tmem_ld_fence(vb);
+#pragma unroll
+          for (int c = 0; c < NCH; c += 2) {
+            if (c + 2 >= NCH) {
+              // every column of this accumulator is in registers: release it
+              tc_fence_before();
+              mbar_arrive(smem_u32(&cs->acc_empty[ab]));
+            }
+            epi_chunk<FP8, H, COLS>(c, va, wsrc, acc);
+            if (c + 2 < NCH) tmem_ld32(taddr + (c + 2) * 32, va);
+            epi_chunk<FP8, H, COLS>(c + 1, vb, wsrc, acc);
+            if (c + 2 < NCH) {
+              tmem_ld32(taddr + (c + 3) * 32, vb);
+              tmem_ld_wait();
+              tmem_ld_fence(va);
+              tmem_ld_fence(vb);
+            }
           }
-          // every column of this accumulator is in registers: release it
-          tc_fence_before();
-          mbar_arrive(smem_u32(&cs->acc_empty[ab]));
           ++acc_it;
-          epi_chunk<H, HALF>(HALF / 32 - 2, va, w4, acc);
-          epi_chunk<H, HALF>(HALF / 32 - 1, vb, w4, acc);
           float skj = 1.0f;
           if (FP8) {
             const int j = u.kbeg + i * kM + kl;
             skj = j < sp.T ? p.s_k[(int64_t)u.b * sp.T + j] : 0.0f;
           }
-          float* st = strip + (size_t)slot * QT * CS + (size_t)half * QH * CS + pos + kl;
+          float* st = strip + (size_t)slot * QT * CS + (size_t)cb * QH * CS + pos + kl;
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql) {
             float s = 0.0f;
@@ -564,43 +576,50 @@ cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap&
 static int strip_max(int QT);
 
 // Shared-memory plan for one MMA width NQ: the query tile (NQ rows), NST
-// key-tile stages, a ring of NSL score strips of CS keys per query (cs_req and
-// nsl_req > 0 fix them), the selection pools (cap keys per query) and the small
-// control block.  Candidates are ranked lexicographically: a pool of at least
-// 1.5K keys first, then enough stages (below), then strips of 512 keys, then
-// the larger pool up to 4K keys (a prune's cost per accepted key falls as
-// cap / (cap - 1.2K)), then more strip slots, then more stages.  Measured on
-// the V4-Flash-shaped step, pool room beats a third stage and extra slots.
+// key-tile ring slots of one K-block each (kM keys x one swizzle span: a
+// whole key tile when a row fits one span, half of one for bf16 at d_I =
+// 128), a ring of NSL score strips of CS keys per query (cs_req and nsl_req >
+// 0 fix them), the selection pools (cap keys per query), the FP8 weight copy
+// and the small control block.  Candidates are ranked lexicographically: a
+// pool of at least 1.5K keys first, then strips of 512 keys, then enough ring
+// slots (below), then the larger pool up to 4K keys (a prune's cost per
+// accepted key falls as cap / (cap - 1.2K)), then more strip slots, then
+// more ring slots.  Measured with S = 262,144 and top-2048, the 512-key strip
+// with one key tile in the ring beats a deeper ring with 128-key strips.
 static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ, int cs_req,
                               int nsl_req) {
   ScorePlan best{};
   best.ok = false;
   const int esz = fp8 ? 1 : 2;
   const int QT = NQ / H;
-  const size_t q_bytes = (size_t)NQ * D * esz;
-  const size_t kc_bytes = (size_t)kM * D * esz;
-  const size_t fixed = 1024 /* alignment slack */ + q_bytes + sizeof(float) * kEpiWarps * kHalfN +
+  const int row_bytes = D * esz;
+  const int sw = row_bytes >= 128 ? 128 : row_bytes;
+  const int kblocks = row_bytes / sw;                  // ring slots per key tile
+  const size_t q_bytes = (size_t)NQ * row_bytes;
+  const size_t slot_bytes = (size_t)kM * sw;
+  const size_t fixed = 1024 /* alignment slack */ + q_bytes +
+                       (fp8 ? sizeof(float) * kEpiWarps * (NQ / 2) : 0) /* FP8 weight copy */ +
                        sizeof(ScoreCtlSmem);
   const int cap_min = ((K + 64 + 31) / 32) * 32;
   const int cap_max = std::max(cap_min, 4 * K);
   const int cs_max = strip_max(QT);
-  // key-tile stages wanted: a full-width tile's MMA (1024 cycles at the
-  // dense rate) hides a tile load from L2 with two stages; a half-width
-  // tile's takes half as long and needs three
-  const int min_nst = NQ == kN ? 2 : 3;
+  // ring slots wanted: a full-width tile's MMA (1024 cycles at the dense
+  // rate) hides the next tile's loads from L2 with two tiles in the ring; a
+  // half-width tile's takes half as long and wants three
+  const int min_slots = (NQ == kN ? 2 : 3) * kblocks;
   long best_score[6] = {-1, -1, -1, -1, -1, -1};
-  for (int nst = 2; nst <= 6; ++nst) {
+  for (int nst = kblocks; nst <= 8; ++nst) {
     for (int cs = 128; cs <= cs_max; cs <<= 1) {
       if (cs_req > 0 && cs != cs_req) continue;
       for (int nsl = 2; nsl <= kMaxSlots; ++nsl) {
         if (nsl_req > 0 && nsl != nsl_req) continue;
-        const size_t used = fixed + nst * kc_bytes + sizeof(float) * (size_t)nsl * QT * cs;
+        const size_t used = fixed + nst * slot_bytes + sizeof(float) * (size_t)nsl * QT * cs;
         if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
         int cap = cap_min;
         while (cap + 32 <= cap_max && used + sel_state_bytes(QT, cap + 32) <= (size_t)max_smem)
           cap += 32;
-        const long sc[6] = {std::min(cap, (3 * K) / 2), std::min(nst, min_nst), std::min(cs, 512),
-                            std::min(cap, 4 * K), nsl, nst};
+        const long sc[6] = {std::min(cap, (3 * K) / 2), std::min(cs, 512),
+                            std::min(nst, min_slots), std::min(cap, 4 * K), nsl, nst};
         bool better = false;
         for (int i = 0; i < 6; ++i) {
           if (sc[i] != best_score[i]) {
@@ -625,21 +644,23 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
   return best;
 }
 
-// The full-width tile (N = 256: 256/H_I queries) is used when its pools can
-// hold 1.5K keys per query; otherwise, for large top-k, the half-width tile
-// (N = 128) halves the queries per tile and so doubles each query's pool,
-// which keeps pruning rare, at the price of reading each key tile from shared
-// memory for half as many columns.
 static int strip_max(int QT) { return std::min(1024, std::max(128, 4096 / QT)); }
 
+// The full-width tile (N = 256: 256/H_I queries) is used when its pools can
+// hold 1.5K keys per query: its MMA reads each key tile from shared memory
+// for twice the columns of the half-width tile (N = 128), whose operand
+// traffic and key-tile stream from L2 cap it well below the dense rate.  For
+// larger top-k the half-width tile halves the queries per tile and so
+// doubles each query's pool, which keeps pruning rare.
 ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req) {
-  ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
+  const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
   if (full.ok && full.cap >= (3 * K) / 2) return full;
   ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
   if (half.ok && (!full.ok || half.cap > full.cap)) return half;
-  if (!full.ok)
-    full.err = (cs_req > strip_max(kN / H) && cs_req > strip_max(kN / 2 / H)) ? 2 : 1;
-  return full;
+  if (full.ok) return full;
+  half.ok = false;
+  half.err = (cs_req > strip_max(kN / H) && cs_req > strip_max(kN / 2 / H)) ? 2 : 1;
+  return half;
 }
 
 }  // namespace si

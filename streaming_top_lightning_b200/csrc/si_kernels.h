@@ -14,6 +14,8 @@ struct ScoreParams {
   SelParams sel;
   UnitGrid ug;
   const float* w;      // [B*S, H] fp32 head weights
+  const float* w_tail; // bf16: [QT, H] copy of the last batch's last query tile's
+                       // rows of w, zero past S (read instead of w by that tile)
   const float* s_q;    // FP8 only: [B*S, H] query row scales
   const float* s_k;    // FP8 only: [B*T] key row scales
   int* counter;        // shared unit counter; this launch's ids start at ug.id_base

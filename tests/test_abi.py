@@ -84,15 +84,16 @@ def test_noalloc_size_check_comes_first(lib):
 
 def test_row_finish_option(lib):
     # rows finished in the fused kernel need no partial lists: the workspace
-    # is the unit counter alone, whatever the problem size
+    # is the unit counter and one query tile's weights (256 columns of fp32,
+    # for a last tile that S leaves partial), whatever the problem size
     for B, S, H, D, k in [(1, 262144, 64, 128, 2048), (64, 65536, 8, 64, 64)]:
         o = _lib.SiOptions(0, 0, 0, 0, 0)
         o.row_finish = 1
         rc, n = _ws(lib, B, S, H, D, 4, k, o)
-        assert rc == 0 and 0 < n <= 256
+        assert rc == 0 and 0 < n <= 256 + 1024
         o.row_finish = 2
         rc, n2 = _ws(lib, B, S, H, D, 4, k, o)
-        assert rc == 0 and n2 > 256
+        assert rc == 0 and n2 > 256 + 1024
     o = _lib.SiOptions(0, 0, 0, 0, 0)
     o.row_finish = 3
     assert _ws(lib, 1, 16384, 64, 128, 4, 512, o)[0] == -8
@@ -128,10 +129,10 @@ def test_plan_query(lib):
     assert p.smem_bytes <= 227 * 1024
     rc, n = _ws(lib, 1, 16384, 64, 128, 4, 512)
     assert rc == 0 and p.workspace_bytes <= n
-    # top-2048 takes the half-width tile (two queries per tile at H_I = 64);
+    # top-2048 keeps the full-width tile (its pools still hold 1.5K keys);
     # its 2624-key lists at S = 262,144 need eleven query blocks
     rc, p = _plan(lib, 1, 262144, 64, 128, 4, 2048)
-    assert rc == 0 and (p.queries_per_tile, p.mma_n, p.query_blocks, p.launches) == (2, 128, 11,
+    assert rc == 0 and (p.queries_per_tile, p.mma_n, p.query_blocks, p.launches) == (4, 256, 11,
                                                                                       22)
     assert p.pool_keys >= 3 * 2048 // 2
     # chunked: score + merge per block and the row sort above k = 512
@@ -140,7 +141,8 @@ def test_plan_query(lib):
     assert rc == 0 and (p.key_chunks, p.query_blocks, p.launches) == (8, 6, 13)
     # errors: topk above the shape's limit, a strip above the tile's limit,
     # bad dims and a bad fp8 flag
-    assert _plan(lib, 1, 4096, 8, 128, 4, 1024)[0] == -3
+    assert _plan(lib, 1, 4096, 8, 128, 4, 1056)[0] == 0
+    assert _plan(lib, 1, 4096, 8, 128, 4, 1057)[0] == -3
     o = _lib.SiOptions(0, 0, 0, 0, 0)
     o.key_tile = 1024
     assert _plan(lib, 1, 4096, 8, 128, 4, 64, opts=o)[0] == -8   # 32 queries: strips <= 128

@@ -61,9 +61,9 @@ def test_half_width_tiles(S, H, D, k):
 
 
 def test_topk_above_the_shape_limit_is_rejected():
-    # with eight heads a 256-column query tile holds 32 queries; their pools
-    # cannot hold top-1024 candidates each
-    sh = synth.small(1, 512, 4, 8, 128, 1024, seed=1)
+    # with eight heads a 128-column query tile holds 16 queries; their pools
+    # hold top-1056 candidates each at d_I = 128, not top-1057
+    sh = synth.small(1, 512, 4, 8, 128, 1057, seed=1)
     q, w, kc = _gpu.inputs(sh, seed=1)
     with pytest.raises(stl.StreamIndexError) as e:
         _gpu.run_bf16(sh, q, w, kc)

@@ -582,10 +582,13 @@ static int strip_max(int QT);
 // 0 fix them), the selection pools (cap keys per query), the FP8 weight copy
 // and the small control block.  Candidates are ranked lexicographically: a
 // pool of at least 1.5K keys first, then strips of 512 keys, then enough ring
-// slots (below), then the larger pool up to 4K keys (a prune's cost per
-// accepted key falls as cap / (cap - 1.2K)), then more strip slots, then
-// more ring slots.  Measured with S = 262,144 and top-2048, the 512-key strip
-// with one key tile in the ring beats a deeper ring with 128-key strips.
+// slots (below), then a third strip slot, then the larger pool up to 4K keys
+// (a prune's cost per accepted key falls as cap / (cap - 1.2K)), then more
+// strip slots, then more ring slots.  Measured with S = 262,144 and
+// top-2048, the 512-key strip with one key tile in the ring beats a deeper
+// ring with 128-key strips, and a third strip slot (it absorbs the
+// selection's uneven pace: a prune holds one query's warp for several
+// strips' worth of MMA time) beats the 256 pool keys it costs by 3%.
 static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int NQ, int cs_req,
                               int nsl_req) {
   ScorePlan best{};
@@ -607,7 +610,7 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
   // rate) hides the next tile's loads from L2 with two tiles in the ring; a
   // half-width tile's takes half as long and wants three
   const int min_slots = (NQ == kN ? 2 : 3) * kblocks;
-  long best_score[6] = {-1, -1, -1, -1, -1, -1};
+  long best_score[7] = {-1, -1, -1, -1, -1, -1, -1};
   for (int nst = kblocks; nst <= 8; ++nst) {
     for (int cs = 128; cs <= cs_max; cs <<= 1) {
       if (cs_req > 0 && cs != cs_req) continue;
@@ -618,17 +621,18 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
         int cap = cap_min;
         while (cap + 32 <= cap_max && used + sel_state_bytes(QT, cap + 32) <= (size_t)max_smem)
           cap += 32;
-        const long sc[6] = {std::min(cap, (3 * K) / 2), std::min(cs, 512),
-                            std::min(nst, min_slots), std::min(cap, 4 * K), nsl, nst};
+        const long sc[7] = {std::min(cap, (3 * K) / 2), std::min(cs, 512),
+                            std::min(nst, min_slots), std::min(nsl, 3),
+                            std::min(cap, 4 * K), nsl, nst};
         bool better = false;
-        for (int i = 0; i < 6; ++i) {
+        for (int i = 0; i < 7; ++i) {
           if (sc[i] != best_score[i]) {
             better = sc[i] > best_score[i];
             break;
           }
         }
         if (better) {
-          for (int i = 0; i < 6; ++i) best_score[i] = sc[i];
+          for (int i = 0; i < 7; ++i) best_score[i] = sc[i];
           best.QT = QT;
           best.nq = NQ;
           best.CS = cs;

@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "indexer query-key pairs/sec, TFLOPS vs B200 peak, peak HBM GB at 1 GPU"
+METRIC_DECODE = "decode indexer query-key pairs/sec, HBM GB/s vs B200 peak"
 UNIT = "pairs/s"
 KERNEL_SRC = os.path.join(ROOT, "streaming_top_lightning_b200", "csrc", "k_score_topk.cu")
 
@@ -495,13 +496,230 @@ def finish(args, sh, ranks, P, K, total_ms, launch_ms, e2e_ms, Ke, h2d, d2h, pea
     return 0
 
 
+# --------------------------------------------------------------------------- decode
+
+
+def decode_pairs(ds) -> int:
+    """Visible query-key pairs of one decode step (all sequences)."""
+    pos = ds.t0 + np.arange(ds.S_q, dtype=np.int64)
+    return int(np.minimum(ds.T, (pos + 1) // ds.seq.m).sum()) * ds.seq.B
+
+
+def decode_config(ds, args):
+    sh = ds.seq
+    kc_bytes = sh.B * ds.T * sh.D * 2
+    return {"workload": ds.name, "B": sh.B, "S_q": ds.S_q, "t0": ds.t0, "T": ds.T, "m": sh.m,
+            "H_I": sh.H, "d_I": sh.D, "topk": sh.topk, "key_chunk": args.key_chunk or
+            "library choice", "score_path": "bf16", "pairs_per_step": decode_pairs(ds),
+            "l2": f"inputs larger than L2: {kc_bytes / 1e6:.0f} MB of keys read per step",
+            "parallelism": f"replicas x{args.gpus} (independent problems)"}
+
+
+def run_decode_reference(args, ds):
+    import oracle
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    q, w, kc = synth.gen_decode(ds)
+    nb = 1
+    per_step = max(0.2, 120.0 / max(1, args.steps + args.warmup))
+    while True:  # sequences per sample, sized once (untimed) to the per-step budget
+        t = time.perf_counter()
+        oracle.indexer_decode(q[:nb], w[:nb], kc[:nb], ds.t0, ds.seq.m, ds.seq.topk)
+        dt = time.perf_counter() - t
+        if dt >= per_step * 0.5 or nb >= ds.seq.B:
+            break
+        nb = min(ds.seq.B, max(nb * 2, int(nb * per_step / max(dt, 1e-3))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        oracle.indexer_decode(q[:nb], w[:nb], kc[:nb], ds.t0, ds.seq.m, ds.seq.topk)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    pairs = decode_pairs(ds) * nb // ds.seq.B
+    value = pairs / float(statistics.median(times))
+    desc = f"{nb} of the {ds.seq.B} sequences of {ds.name}, every visible key scored in fp64"
+    line = {"impl": "reference", "metric": METRIC_DECODE, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * decode_pairs(ds) / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": decode_config(ds, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, ds):
+    """A decode step: the newest query of each of B sequences against the
+    keys compressed so far (resident on the GPU, as a KV cache is).  The
+    score kernel reads every visible key once, so its bound is HBM."""
+    import torch
+    import torch.distributed as dist
+
+    import streaming_top_lightning_b200 as stl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ranks = Ranks(dist, world, rank, dev)
+    sh = ds.seq
+    q, w, kc = synth.gen_decode(ds, seed=rank)
+    q_h = torch.from_numpy(q.view(np.int16)).pin_memory()
+    w_h = torch.from_numpy(w).pin_memory()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    torch.cuda.reset_peak_memory_stats()
+    kc_d = torch.from_numpy(kc.view(np.int16)).to(dev).view(torch.bfloat16)
+    q_d = q_h.to(dev).view(torch.bfloat16)
+    w_d = w_h.to(dev)
+    opts = stl.options(key_chunk=args.key_chunk)
+    ws = torch.empty(max(16, stl.decode_workspace_size(sh.B, ds.S_q, ds.t0, ds.T, sh.H, sh.D,
+                                                       sh.m, sh.topk, opts)),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty((sh.B, ds.S_q, sh.topk), dtype=torch.int32, device=dev)
+    score = torch.empty((sh.B, ds.S_q, sh.topk), dtype=torch.float32, device=dev)
+    plan = stl.decode_plan(sh.B, ds.S_q, ds.t0, ds.T, sh.H, sh.D, sh.m, sh.topk, opts)
+    stream = torch.cuda.current_stream()
+    K = args.steps
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for lst in kev:
+        for e in lst:
+            e.record(stream)
+    kopts = [stl.options(key_chunk=args.key_chunk, score_event_list=lst) for lst in kev]
+
+    def step(o):
+        stl.indexer_decode(q_d, w_d, kc_d, ds.t0, sh.m, sh.topk, out=(idx, score), opts=o,
+                           workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step(opts)
+    torch.cuda.synchronize()
+    if stl.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    peak_alloc = torch.cuda.max_memory_allocated()
+    free1, _ = torch.cuda.mem_get_info()
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        pass
+    with ClockSampler(uuid) as clk:
+        ranks.barrier()
+        torch.cuda.synchronize()
+        t0e.record(stream)
+        for i in range(K):
+            step(kopts[i])
+        t1e.record(stream)
+        torch.cuda.synchronize()
+        ranks.barrier()
+    if stl.device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+    total_ms = ranks.max_over_ranks(t0e.elapsed_time(t1e))
+    score_ms = statistics.mean(lst[0].elapsed_time(lst[1]) for lst in kev)
+
+    # end to end through the public API: each step's new queries and weights
+    # go host -> device, the selected rows come back; the keys stay resident
+    idx_h = torch.empty(tuple(idx.shape), dtype=torch.int32).pin_memory()
+    score_h = torch.empty(tuple(score.shape), dtype=torch.float32).pin_memory()
+    qe, we = torch.empty_like(q_h, device=dev), torch.empty_like(w_h, device=dev)
+
+    def e2e_step():
+        qe.copy_(q_h, non_blocking=True)
+        we.copy_(w_h, non_blocking=True)
+        stl.indexer_decode(qe.view(torch.bfloat16), we, kc_d, ds.t0, sh.m, sh.topk,
+                           out=(idx, score), opts=opts, workspace=ws)
+        idx_h.copy_(idx, non_blocking=True)
+        score_h.copy_(score, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ranks.barrier()
+    e2e_ms = ranks.max_over_ranks(e0.elapsed_time(e1)) / K
+    assert stl.device_error() == 0
+
+    pairs = decode_pairs(ds)
+    ms_per_step = total_ms / K
+    # algorithmic bytes of the score kernel: every visible key read once, the
+    # queries and weights, and the candidate lists it writes
+    pos = ds.t0 + np.arange(ds.S_q)
+    vis = int(np.minimum(ds.T, (pos.max() + 1) // sh.m))
+    kc_bytes = sh.B * vis * sh.D * 2
+    qw_bytes = sh.B * ds.S_q * sh.H * (sh.D * 2 + 4)
+    lists = (sh.B * plan["key_chunks"] * plan["queries_per_tile"] * plan["partial_len"] * 8
+             if plan["key_chunks"] > 1 else 0)
+    alg = kc_bytes + qw_bytes + lists
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    achieved = alg / (score_ms / 1e3) / 1e9
+    h2d = q_h.numel() * 2 + w_h.numel() * 4
+    d2h = idx_h.numel() * 4 + score_h.numel() * 4
+    line = {
+        "metric": METRIC_DECODE, "value": ranks.job_value(pairs, ms_per_step), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; distributions of the workload recipe)",
+        "config": decode_config(ds, args),
+        "step_gbs": alg / (ms_per_step / 1e3) / 1e9,
+        "peak_hbm_gb": peak_alloc / 1e9, "hbm_in_use_delta_gb": (free0 - free1) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "kernel": "k_score_topk",
+                     "peak_source": f"{peak_src} hbm_gbs",
+                     "algorithmic_bytes_per_step": alg,
+                     "score_kernel_ms_per_step": score_ms,
+                     "timing": "CUDA events recorded by the library around the score-kernel "
+                               "launch"},
+        "plan": {k: plan[k] for k in ("queries_per_tile", "mma_n", "key_tile", "stages",
+                                      "strip_slots", "pool_keys", "key_chunks", "launches")},
+        "e2e": {"value": ranks.job_value(pairs, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "resident": "the keys (a KV cache stays on the GPU between steps)"},
+        "gpu_launches": K * plan["launches"],
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+
+        nb = max(1, min(sh.B, 4))
+        t = time.perf_counter()
+        oracle.indexer_decode(q[:nb], w[:nb], kc[:nb], ds.t0, sh.m, sh.topk)
+        secs = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": pairs * nb / sh.B / secs, "unit": UNIT,
+                                "cores": oracle.threads(), "kind": "oracle",
+                                "sample": f"{nb} of the {sh.B} sequences", "seconds": secs}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="long_s256k", choices=sorted(synth.SHAPES))
+    ap.add_argument("--workload", default="long_s256k",
+                    choices=sorted(synth.SHAPES) + sorted(synth.DECODE_SHAPES))
     ap.add_argument("--key-chunk", type=int, default=0)
     ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
                     help="1: rows finished in the fused kernel; 2: by the merge kernel; "
@@ -516,6 +734,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
+    if args.workload in synth.DECODE_SHAPES:
+        ds = synth.DECODE_SHAPES[args.workload]
+        if args.fp8 or args.topk or args.key_tile or args.strip_slots or args.row_finish:
+            ap.error("decode workloads take only --key-chunk among the workload options")
+        return (run_decode_reference if args.impl == "reference" else run_decode)(args, ds)
     sh = synth.shape(args.workload)
     if args.topk:
         sh = synth.shape(args.workload, topk=args.topk)

@@ -34,7 +34,8 @@
  *    aligned.  The selection keeps a candidate pool per query of a query
  *    tile in shared memory, so with few heads (many queries per tile) the
  *    largest topk is lower: bf16 H_I=8: 1056 (d_I=128), 1312 (d_I=64);
- *    FP8 H_I=8: 1280 (d_I=128), 1408 (d_I=64); 2048 otherwise.  A larger topk returns SI_ERR_TOPK.
+ *    FP8 H_I=8: 1280 (d_I=128), 1408 (d_I=64); 2048 otherwise.  A larger
+ *    topk returns SI_ERR_TOPK.
  */
 #ifndef STREAMINDEX_H
 #define STREAMINDEX_H
@@ -234,6 +235,45 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
 int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B, int S, int H_I,
                             int d_I, int m, int topk, int32_t* out_idx, float* out_score,
                             void* stream);
+
+/* ---- decode ------------------------------------------------------------ */
+
+/*
+ * si_indexer_decode: the indexer step for the newest queries of sequences
+ * whose compressed keys so far are given.  The abstract describes the step
+ * for a whole sequence (every query against the keys it can see); decoding
+ * scores only the queries of the tokens just produced, against the keys
+ * compressed so far, so the result is the same formula with each query's
+ * sequence position in place of t:
+ *   query i of batch b sits at position t = t0 + i (0 <= i < S_q, the same
+ *   t0 in every batch) and sees the first V = min(T, floor((t+1)/m)) keys.
+ * A query row of a decode call therefore equals row t0 + i of si_indexer_topk
+ * on a sequence whose keys are kc: a caller that appends one compressed key
+ * per m tokens passes the grown kc and the new position each step.
+ *   q         bf16 [B,S_q,H_I,d_I]   queries at positions t0 .. t0+S_q-1
+ *   w         fp32 [B,S_q,H_I]       their head weights
+ *   kc        bf16 [B,T,d_I]         compressed keys; keys past a query's V
+ *                                    are never used (kc may be a buffer with
+ *                                    room for more keys)
+ *   out_idx   int32 [B,S_q,topk], out_score fp32 [B,S_q,topk]: as si_indexer_topk.
+ * Limits: B, S_q, T, m >= 1; t0 >= 0 and t0 + S_q < 2^31; B*T < 2^31; H_I,
+ * d_I, topk and alignment as si_indexer_topk (S need not be a multiple of m).
+ * With few query tiles the keys of a tile are split into chunks so that the
+ * work spreads over every SM (options.key_chunk > 0 fixes the chunk), and the
+ * chunks' candidate lists are merged.  Workspace: caller-provided, at least
+ * si_indexer_decode_workspace_size bytes.  bf16 operands only.
+ */
+int si_indexer_decode(const void* q, const float* w, const void* kc, int B, int S_q, int t0, int T,
+                      int H_I, int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                      const si_options* opt, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace si_indexer_decode needs. */
+int si_indexer_decode_workspace_size(int B, int S_q, int t0, int T, int H_I, int d_I, int m,
+                                     int topk, const si_options* opt, size_t* bytes);
+
+/* The plan si_indexer_decode would run (see si_indexer_topk_plan). */
+int si_indexer_decode_plan(int B, int S_q, int t0, int T, int H_I, int d_I, int m, int topk,
+                           const si_options* opt, si_plan_info* out);
 
 /* ---- diagnostics ------------------------------------------------------ */
 

@@ -194,6 +194,30 @@ def row_absmax_rows(q_rows, w_rows, kc, S: int, m: int, rows, lib=None):
     return out
 
 
+def decode_rows(B: int, S_q: int, t0: int, T: int, m: int, lib=None):
+    """Rows of the row functions above that stand for the decode queries:
+    query i of batch b, at sequence position t0 + i, sees V = min(T,
+    floor((t0+i+1)/m)) keys, which is what the row at position min(t0+i,
+    m*T-1) of a sequence of m*T tokens (T keys) sees.  Returns (S, rows) to
+    pass as the row functions' S and rows, with kc [B,T,D].  (lib: unused;
+    present so every function of the module takes it.)"""
+    S = m * T
+    pos = np.minimum(t0 + np.arange(S_q, dtype=np.int64), S - 1)
+    rows = (np.arange(B, dtype=np.int64)[:, None] * S + pos[None, :]).reshape(-1)
+    return S, rows
+
+
+def indexer_decode(q, w, kc, t0: int, m: int, k: int, lib=None):
+    """Decode oracle: q [B,S_q,H,D] bf16 bits and w [B,S_q,H] at positions
+    t0 .. t0+S_q-1 against kc [B,T,D].  Returns (idx, score, absmax) with one
+    row per query, batch-major."""
+    q, w = _c(q, np.uint16), _c(w, np.float32)
+    B, S_q, H, D = q.shape
+    S, rows = decode_rows(B, S_q, t0, kc.shape[1], m)
+    return indexer_topk_rows_absmax(q.reshape(B * S_q, H, D), w.reshape(B * S_q, H), kc, S, m, k,
+                                    rows, lib=lib)
+
+
 def topk_scores(X, m: int, k: int, rows=None, lib=None):
     """Selection alone on given fp32 scores X [B,S,T].
     Returns (idx [n,k] int32, score [n,k] float32 carrying the input bit patterns)."""
@@ -264,4 +288,5 @@ def score_keys_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, rows,
 _API = {name: globals()[name] for name in (
     "threads", "visible", "indexer_topk", "indexer_topk_rows", "indexer_topk_rows_absmax",
     "score_keys_rows", "row_absmax_rows", "topk_scores", "e4m3_decode", "e4m3_encode",
-    "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows")}
+    "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows", "decode_rows",
+    "indexer_decode")}

@@ -57,6 +57,25 @@ def topk(q, w, kc, m: int, k: int):
     return out_idx, out_sc
 
 
+def topk_decode(q, w, kc, m: int, k: int, t0: int):
+    """Decode form: query i of batch b sits at sequence position t0 + i and
+    sees the keys j with (j+1)*m - 1 <= t0 + i (all T of them once the
+    position is past the last key).  q [B,S_q,H,D], w [B,S_q,H], kc [B,T,D].
+    Returns (idx, score) as in topk()."""
+    B, S = q.shape[0], q.shape[1]
+    T = kc.shape[1]
+    out_idx, out_sc = [], []
+    for b in range(B):
+        for i in range(S):
+            V = visible_count(t0 + i, T, m)
+            pairs = [(score(q, w, kc, b, i, j), j) for j in range(V)]
+            pairs.sort(key=lambda p: (-p[0], p[1]))
+            sel = pairs[:k]
+            out_idx.append([j for _, j in sel] + [-1] * (k - len(sel)))
+            out_sc.append([s for s, _ in sel] + [None] * (k - len(sel)))
+    return out_idx, out_sc
+
+
 def e4m3_value(code: int) -> Fraction:
     """Exact value of an OCP E4M3 code (bias 7, 3 mantissa bits, exponent
     field 0 subnormal), written out from the format's definition."""

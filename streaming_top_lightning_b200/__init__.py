@@ -149,6 +149,53 @@ def indexer_topk(q, w, kc, m: int, topk: int, *, out=None, opts: SiOptions | Non
     return idx, score
 
 
+def decode_workspace_size(B: int, S_q: int, t0: int, T: int, H: int, D: int, m: int, topk: int,
+                          opts: SiOptions | None = None) -> int:
+    n = ctypes.c_size_t(0)
+    lib = _lib.load()
+    _lib.check("si_indexer_decode_workspace_size",
+               lib.si_indexer_decode_workspace_size(B, S_q, t0, T, H, D, m, topk,
+                                                    ctypes.byref(opts) if opts else None,
+                                                    ctypes.byref(n)))
+    return n.value
+
+
+def decode_plan(B: int, S_q: int, t0: int, T: int, H: int, D: int, m: int, topk: int,
+                opts: SiOptions | None = None) -> dict:
+    """The plan si_indexer_decode would run (tile shape, key chunks, launches)."""
+    info = SiPlanInfo()
+    lib = _lib.load()
+    _lib.check("si_indexer_decode_plan",
+               lib.si_indexer_decode_plan(B, S_q, t0, T, H, D, m, topk,
+                                          ctypes.byref(opts) if opts else None,
+                                          ctypes.byref(info)))
+    return info.as_dict()
+
+
+def indexer_decode(q, w, kc, t0: int, m: int, topk: int, *, out=None,
+                   opts: SiOptions | None = None, workspace=None, stream=None):
+    """Top-k compressed keys for the queries at sequence positions t0 ..
+    t0 + S_q - 1 (q [B,S_q,H,D] bf16, w [B,S_q,H] fp32) against the keys kc
+    [B,T,D] bf16 compressed so far (si_indexer_decode).  Returns (idx, score),
+    each [B,S_q,topk]."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    _need(w, torch.float32, 3, "w")
+    _need(kc, torch.bfloat16, 3, "kc")
+    B, S, H, D = q.shape
+    T = kc.shape[1]
+    idx, score = _outputs(B, S, topk, q.device, out)
+    need = decode_workspace_size(B, S, t0, T, H, D, m, topk, opts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = _lib.load().si_indexer_decode(_ptr(q), _ptr(w), _ptr(kc), B, S, t0, T, H, D, m, topk,
+                                       _ptr(idx), _ptr(score),
+                                       ctypes.byref(opts) if opts else None, _ptr(workspace),
+                                       workspace.numel(), _stream(stream))
+    _lib.check("si_indexer_decode", rc)
+    return idx, score
+
+
 def indexer_topk_noalloc(q, w, kc, m: int, topk: int, *, out=None, stream=None):
     """``indexer_topk`` through the entry point that allocates no device memory
     (its scratch is a fixed array inside the library; see

@@ -23,7 +23,8 @@ EXPORTS = [
     "si_indexer_topk", "si_indexer_topk_workspace_size", "si_indexer_topk_ex",
     "si_indexer_topk_fp8", "si_quantize_fp8_rows", "si_topk_scores", "si_status_string",
     "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc", "si_indexer_topk_plan",
-    "si_role_cycles",
+    "si_role_cycles", "si_indexer_decode", "si_indexer_decode_workspace_size",
+    "si_indexer_decode_plan",
 ]
 
 
@@ -86,6 +87,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.si_get_last_device_error.argtypes = [P]
     lib.si_version.argtypes = []
     lib.si_role_cycles.argtypes = [P, I, I]
+    lib.si_indexer_decode.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, P, OP, P, Z, P]
+    lib.si_indexer_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, I, OP,
+                                                     ctypes.POINTER(Z)]
+    lib.si_indexer_decode_plan.argtypes = [I, I, I, I, I, I, I, I, OP,
+                                           ctypes.POINTER(SiPlanInfo)]
     for name in EXPORTS:
         if name != "si_status_string":
             getattr(lib, name).restype = I

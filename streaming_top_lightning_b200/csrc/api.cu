@@ -96,6 +96,12 @@ void plan_limits(int* max_smem, int* sms) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Keys a query at sequence position t sees: min(T, (t+1)/m).
+int visible_host(int t, int T, int m) {
+  const int v = (int)(((int64_t)t + 1) / m);
+  return v < T ? v : T;
+}
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // 2-D row-major [rows, cols] tensor map with a {box_inner, box_rows} box and
@@ -236,38 +242,96 @@ int plan_status(const ScorePlan& sp) {
   return sp.err == 2 ? SI_ERR_OPTIONS : SI_ERR_TOPK;
 }
 
+// The queries and keys of one call.  Prefill: S queries per batch at
+// positions 0 .. S-1, T = S/m keys, t0 = 0.  Decode: S queries per batch at
+// positions t0 .. t0+S-1, against T keys.
+struct Problem {
+  int B, S, T, t0, m;
+  bool decode;
+};
+
 int check_common(int B, int S, int m, int topk) {
   if (B < 1 || S < 1 || m < 1 || S % m != 0) return SI_ERR_DIM;
   if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
   return SI_OK;
 }
 
-int check_indexer(const void* q, const void* w, const void* kc, int B, int S, int H, int D, int m,
+// Sizes of a prefill (S % m == 0, T = S/m, t0 = 0) or decode call.
+int check_problem(const Problem& pb, int H, int D, int topk) {
+  if (pb.decode) {
+    if (pb.B < 1 || pb.S < 1 || pb.T < 1 || pb.t0 < 0 || pb.m < 1 ||
+        (int64_t)pb.t0 + pb.S > 0x7FFFFFFF)
+      return SI_ERR_DIM;
+    if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
+  } else {
+    int rc = check_common(pb.B, pb.S, pb.m, topk);
+    if (rc) return rc;
+  }
+  if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
+  if ((int64_t)pb.B * pb.S * H >= ((int64_t)1 << 31)) return SI_ERR_DIM;
+  if ((int64_t)pb.B * pb.T >= ((int64_t)1 << 31)) return SI_ERR_DIM;
+  return SI_OK;
+}
+
+Problem prefill(int B, int S, int m) { return Problem{B, S, m > 0 ? S / m : 0, 0, m, false}; }
+
+// Pointers first, then sizes, then alignment.
+int check_indexer(const void* q, const void* w, const void* kc, const Problem& pb, int H, int D,
                   int topk, const void* oi, const void* os) {
   if (!q || !w || !kc || !oi || !os) return SI_ERR_NULL;
-  int rc = check_common(B, S, m, topk);
+  int rc = check_problem(pb, H, D, topk);
   if (rc) return rc;
-  if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
-  if ((int64_t)B * S * H >= ((int64_t)1 << 31)) return SI_ERR_DIM;
   if (!aligned16(q) || !aligned16(w) || !aligned16(kc) || !aligned16(oi) || !aligned16(os))
     return SI_ERR_ALIGN;
   return SI_OK;
 }
 
+// Default key chunk of a decode call (0: one chunk per query tile).  With
+// fewer query tiles than SMs a tile's keys are split into chunks, so that
+// (tile, chunk) units fill the GPU; the chunk count minimises the rounds of
+// units times the chunk length, charging each chunk about 256 keys' worth of
+// fixed cost (its query-tile load and its partial list).
+int decode_key_chunk(const Problem& pb, int QT, int sms) {
+  const int64_t tiles = (int64_t)pb.B * ((pb.S + QT - 1) / QT);
+  const int vmax = visible_host(pb.t0 + pb.S - 1, pb.T, pb.m);
+  if (vmax <= 128 || tiles >= sms) return 0;
+  int best_c = 0;
+  int64_t best_cost = -1;
+  for (int nch = 1; nch <= 64; ++nch) {
+    const int c = ((vmax + nch - 1) / nch + 127) / 128 * 128;
+    const int64_t n = (vmax + c - 1) / c;
+    const int64_t rounds = (tiles * n + sms - 1) / sms;
+    const int64_t cost = rounds * (c + 256);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_c = n == 1 ? 0 : c;
+    }
+  }
+  return best_c;
+}
+
+Plan plan_for(const Problem& pb, int K, int QT, int H, const Opts& o, int sms) {
+  Opts oc = o;
+  if (pb.decode && oc.key_chunk == 0) oc.key_chunk = decode_key_chunk(pb, QT, sms);
+  return make_plan(pb.B, pb.S, pb.T, K, QT, H, oc);
+}
+
 int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const void* kc,
-                const float* s_k, int B, int S, int H, int D, int m, int K, int32_t* out_idx,
+                const float* s_k, const Problem& pb, int H, int D, int K, int32_t* out_idx,
                 float* out_score, const si_options* opt, void* ws, size_t ws_bytes,
                 cudaStream_t stream) {
-  int rc = check_indexer(q, w, kc, B, S, H, D, m, K, out_idx, out_score);
+  const int B = pb.B, S = pb.S, m = pb.m;
+  int rc = check_indexer(q, w, kc, pb, H, D, K, out_idx, out_score);
   if (rc) return rc;
   if (fp8 && (!s_q || !s_k)) return SI_ERR_NULL;
   Opts o;
   if ((rc = read_opts(opt, &o))) return rc;
   DevInfo* dev;
   if ((rc = dev_info(&dev))) return rc;
-  const ScorePlan sp_plan = plan_score(fp8, D, H, K, dev->max_smem, o.key_tile, o.strip_slots);
+  const ScorePlan sp_plan =
+      plan_score(fp8, D, H, K, dev->max_smem, o.key_tile, o.strip_slots, pb.S);
   if ((rc = plan_status(sp_plan))) return rc;  // pools of this topk do not fit, or key_tile
-  const Plan pl = make_plan(B, S, S / m, K, sp_plan.QT, H, o);
+  const Plan pl = plan_for(pb, K, sp_plan.QT, H, o, dev->sms);
   if (!ws || ws_bytes < pl.ws_bytes()) return SI_ERR_WORKSPACE;
   if (!aligned16(ws)) return SI_ERR_ALIGN;
 
@@ -308,11 +372,11 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   for (int blk = 0; blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, 1};
+    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, 1, pb.t0};
     ScoreParams p{};
     p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
                       sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,
-                      out_idx, out_score, partial, pl.final_rows};
+                      out_idx, out_score, partial, pl.final_rows, pb.t0};
     p.ug = ug;
     p.w = w;
     p.w_tail = w_tail;
@@ -353,18 +417,17 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   return SI_OK;
 }
 
-int workspace_for(bool fp8, int S, int B, int H, int D, int m, int K, const si_options* opt,
-                  size_t* bytes) {
-  int rc = check_common(B, S, m, K);
+int workspace_for(const Problem& pb, int H, int D, int K, const si_options* opt, size_t* bytes) {
+  int rc = check_problem(pb, H, D, K);
   if (rc) return rc;
-  if (!(H == 8 || H == 16 || H == 32 || H == 64) || !(D == 64 || D == 128)) return SI_ERR_DIM;
   Opts o;
   if ((rc = read_opts(opt, &o))) return rc;
+  int max_smem = 0, sms = 0;
+  plan_limits(&max_smem, &sms);
   // the larger need of the two query-tile widths the score plan may choose
-  const Plan full = make_plan(B, S, S / m, K, 256 / H, H, o);
-  const Plan half = make_plan(B, S, S / m, K, 128 / H, H, o);
+  const Plan full = plan_for(pb, K, 256 / H, H, o, sms);
+  const Plan half = plan_for(pb, K, 128 / H, H, o, sms);
   *bytes = std::max(full.ws_bytes(), half.ws_bytes());
-  (void)fp8;
   return SI_OK;
 }
 
@@ -399,8 +462,7 @@ int noalloc_scratch(void** out) {
 static int host_tile_vmax(const UnitGrid& u, int g) {
   int t = g * u.QT + u.QT - 1;
   if (t > u.S - 1) t = u.S - 1;
-  const int v = (t + 1) / u.m;
-  return v < u.T ? v : u.T;
+  return visible_host(u.t0 + t, u.T, u.m);
 }
 
 int host_tile_chunks(const UnitGrid& u, int g) {
@@ -419,6 +481,38 @@ int host_count_units(const UnitGrid& u) {
 }  // namespace si
 
 using namespace si;
+
+// The plan of a prefill or decode call, as si_plan_info.
+static int plan_info(const Problem& pb, int H, int D, int topk, int fp8, const si_options* opt,
+              si_plan_info* out) {
+  if (!out) return SI_ERR_NULL;
+  int rc = check_problem(pb, H, D, topk);
+  if (rc) return rc;
+  if (fp8 < 0 || fp8 > 1) return SI_ERR_OPTIONS;
+  Opts o;
+  if ((rc = read_opts(opt, &o))) return rc;
+  int max_smem = 0, sms = 0;
+  plan_limits(&max_smem, &sms);
+  const ScorePlan sp =
+      plan_score(fp8 != 0, D, H, topk, max_smem, o.key_tile, o.strip_slots, pb.S);
+  if ((rc = plan_status(sp))) return rc;
+  const Plan pl = plan_for(pb, topk, sp.QT, H, o, sms);
+  si_plan_info r{};
+  r.queries_per_tile = sp.QT;
+  r.mma_n = sp.nq;
+  r.key_tile = sp.CS;
+  r.stages = sp.nst;
+  r.strip_slots = sp.nslot;
+  r.pool_keys = sp.cap;
+  r.partial_len = pl.L;
+  r.key_chunks = pl.nch_max;
+  r.query_blocks = pl.n_blocks;
+  r.launches = plan_launches(pl, topk);
+  r.workspace_bytes = pl.ws_bytes();
+  r.smem_bytes = sp.smem;
+  *out = r;
+  return SI_OK;
+}
 
 extern "C" {
 
@@ -443,45 +537,18 @@ const char* si_status_string(int s) {
 int si_indexer_topk_workspace_size(int B, int S, int H_I, int d_I, int m, int topk,
                                    const si_options* opt, size_t* bytes) {
   if (!bytes) return SI_ERR_NULL;
-  return workspace_for(false, S, B, H_I, d_I, m, topk, opt, bytes);
+  return workspace_for(prefill(B, S, m), H_I, d_I, topk, opt, bytes);
 }
 
 int si_indexer_topk_plan(int B, int S, int H_I, int d_I, int m, int topk, int fp8,
                          const si_options* opt, si_plan_info* out) {
-  if (!out) return SI_ERR_NULL;
-  int rc = check_common(B, S, m, topk);
-  if (rc) return rc;
-  if (!(H_I == 8 || H_I == 16 || H_I == 32 || H_I == 64) || !(d_I == 64 || d_I == 128))
-    return SI_ERR_DIM;
-  if (fp8 < 0 || fp8 > 1) return SI_ERR_OPTIONS;
-  Opts o;
-  if ((rc = read_opts(opt, &o))) return rc;
-  int max_smem = 0, sms = 0;
-  plan_limits(&max_smem, &sms);
-  const ScorePlan sp = plan_score(fp8 != 0, d_I, H_I, topk, max_smem, o.key_tile, o.strip_slots);
-  if ((rc = plan_status(sp))) return rc;
-  const Plan pl = make_plan(B, S, S / m, topk, sp.QT, H_I, o);
-  si_plan_info r{};
-  r.queries_per_tile = sp.QT;
-  r.mma_n = sp.nq;
-  r.key_tile = sp.CS;
-  r.stages = sp.nst;
-  r.strip_slots = sp.nslot;
-  r.pool_keys = sp.cap;
-  r.partial_len = pl.L;
-  r.key_chunks = pl.nch_max;
-  r.query_blocks = pl.n_blocks;
-  r.launches = plan_launches(pl, topk);
-  r.workspace_bytes = pl.ws_bytes();
-  r.smem_bytes = sp.smem;
-  *out = r;
-  return SI_OK;
+  return plan_info(prefill(B, S, m), H_I, d_I, topk, fp8, opt, out);
 }
 
 int si_indexer_topk_ex(const void* q, const float* w, const void* kc, int B, int S, int H_I,
                        int d_I, int m, int topk, int32_t* out_idx, float* out_score,
                        const si_options* opt, void* workspace, size_t ws_bytes, void* stream) {
-  return run_indexer(false, q, nullptr, w, kc, nullptr, B, S, H_I, d_I, m, topk, out_idx,
+  return run_indexer(false, q, nullptr, w, kc, nullptr, prefill(B, S, m), H_I, d_I, topk, out_idx,
                      out_score, opt, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -490,7 +557,7 @@ int si_indexer_topk(const void* q, const float* w, const void* kc, int B, int S,
   size_t bytes = 0;
   int rc = si_indexer_topk_workspace_size(B, S, H_I, d_I, m, topk, nullptr, &bytes);
   if (rc) return rc;
-  rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score);
+  rc = check_indexer(q, w, kc, prefill(B, S, m), H_I, d_I, topk, out_idx, out_score);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* ws = nullptr;
@@ -505,7 +572,8 @@ int si_indexer_topk_fp8(const void* q8, const float* s_q, const float* w, const 
                         const float* s_k, int B, int S, int H_I, int d_I, int m, int topk,
                         int32_t* out_idx, float* out_score, const si_options* opt,
                         void* workspace, size_t ws_bytes, void* stream) {
-  return run_indexer(true, q8, s_q, w, k8, s_k, B, S, H_I, d_I, m, topk, out_idx, out_score, opt,
+  return run_indexer(true, q8, s_q, w, k8, s_k, prefill(B, S, m), H_I, d_I, topk, out_idx,
+                     out_score, opt,
                      workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -543,7 +611,7 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
     // the fused kernel's selection plan for that shape: same queries per
     // tile, strip length and pool room, hence the same selection steps
     const ScorePlan fp = plan_score(o.plan_fp8 != 0, o.plan_dim, o.plan_heads, topk,
-                                    dev->max_smem, o.key_tile, o.strip_slots);
+                                    dev->max_smem, o.key_tile, o.strip_slots, 0);
     if ((rc = plan_status(fp))) return rc;
     QT = fp.QT;
     CS = fp.CS;
@@ -564,10 +632,10 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   for (int blk = 0; rc == SI_OK && blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base, 0};
+    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base, 0, 0};
     SelParams sp{B,    S,       T,          m,       topk,    QT,     CS,
                  cap,  pl.L,    g_lo,       n_tiles, pl.nch_max, out_idx, out_score,
-                 partial, pl.final_rows};
+                 partial, pl.final_rows, 0};
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -627,14 +695,35 @@ int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B
   si_options opt{};
   opt.scratch_mb = (int)(kNoAllocScratchBytes >> 20) - 1;
   size_t need = 0;
-  int rc = workspace_for(false, S, B, H_I, d_I, m, topk, &opt, &need);
+  int rc = workspace_for(prefill(B, S, m), H_I, d_I, topk, &opt, &need);
   if (rc) return rc;
   if (need > kNoAllocScratchBytes) return SI_ERR_WORKSPACE;  // one query tile does not fit
-  if ((rc = check_indexer(q, w, kc, B, S, H_I, d_I, m, topk, out_idx, out_score))) return rc;
+  if ((rc = check_indexer(q, w, kc, prefill(B, S, m), H_I, d_I, topk, out_idx, out_score)))
+    return rc;
   void* ws = nullptr;
   if ((rc = noalloc_scratch(&ws))) return rc;
-  return run_indexer(false, q, nullptr, w, kc, nullptr, B, S, H_I, d_I, m, topk, out_idx,
+  return run_indexer(false, q, nullptr, w, kc, nullptr, prefill(B, S, m), H_I, d_I, topk, out_idx,
                      out_score, &opt, ws, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ decode
+int si_indexer_decode_workspace_size(int B, int S_q, int t0, int T, int H_I, int d_I, int m,
+                                     int topk, const si_options* opt, size_t* bytes) {
+  if (!bytes) return SI_ERR_NULL;
+  return workspace_for(Problem{B, S_q, T, t0, m, true}, H_I, d_I, topk, opt, bytes);
+}
+
+int si_indexer_decode_plan(int B, int S_q, int t0, int T, int H_I, int d_I, int m, int topk,
+                           const si_options* opt, si_plan_info* out) {
+  return plan_info(Problem{B, S_q, T, t0, m, true}, H_I, d_I, topk, 0, opt, out);
+}
+
+int si_indexer_decode(const void* q, const float* w, const void* kc, int B, int S_q, int t0, int T,
+                      int H_I, int d_I, int m, int topk, int32_t* out_idx, float* out_score,
+                      const si_options* opt, void* workspace, size_t ws_bytes, void* stream) {
+  return run_indexer(false, q, nullptr, w, kc, nullptr, Problem{B, S_q, T, t0, m, true}, H_I, d_I,
+                     topk, out_idx, out_score, opt, workspace, ws_bytes,
+                     static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

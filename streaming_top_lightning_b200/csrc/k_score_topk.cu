@@ -655,11 +655,15 @@ static int strip_max(int QT) { return std::min(1024, std::max(128, 4096 / QT)); 
 // for twice the columns of the half-width tile (N = 128), whose operand
 // traffic and key-tile stream from L2 cap it well below the dense rate.  For
 // larger top-k the half-width tile halves the queries per tile and so
-// doubles each query's pool, which keeps pruning rare.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req) {
+// doubles each query's pool, which keeps pruning rare.  When every batch has
+// no more queries than a half-width tile holds (a decode step), the
+// half-width tile does the same work with half the MMA and epilogue columns.
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req,
+                     int rows) {
+  ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
+  if (half.ok && rows > 0 && rows <= half.QT) return half;
   const ScorePlan full = plan_score_n(fp8, D, H, K, max_smem, kN, cs_req, nsl_req);
   if (full.ok && full.cap >= (3 * K) / 2) return full;
-  ScorePlan half = plan_score_n(fp8, D, H, K, max_smem, kN / 2, cs_req, nsl_req);
   if (half.ok && (!full.ok || half.cap > full.cap)) return half;
   if (full.ok) return full;
   half.ok = false;

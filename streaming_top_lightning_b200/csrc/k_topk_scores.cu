@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
         for (int qi = 0; qi < QT; ++qi) {
           const int t = g * QT + qi;
           if (t >= sp.S) break;
-          const int lim = min(nk, visible_keys(t, sp.T, sp.m) - j0);
+          const int lim = min(nk, visible_keys(sp.t0 + t, sp.T, sp.m) - j0);
           const float* src = X + ((int64_t)b * sp.S + t) * sp.T + j0;
           for (int q = tid; q < lim; q += kLoadThreads) st[(size_t)qi * CS + q] = __ldg(src + q);
         }

@@ -43,7 +43,9 @@ struct ScorePlan {
 
 // cs_req: keys per score strip (128 .. 1024), nsl_req: strip ring slots
 // (2 .. 4); 0 = the planner's choice.
-ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req);
+// rows: queries per batch when known and small (0: many), see k_score_topk.cu
+ScorePlan plan_score(bool fp8, int D, int H, int K, int max_smem, int cs_req, int nsl_req,
+                     int rows);
 
 cudaError_t launch_score_topk(bool fp8, int D, int H, int nq, const CUtensorMap& tm_q,
                               const CUtensorMap& tm_kc, const ScoreParams& p, int grid,

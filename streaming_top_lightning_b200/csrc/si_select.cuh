@@ -47,6 +47,7 @@ struct SelParams {
   uint64_t* partial;   // [B, n_tiles, nch_max, QT, L] candidate keys, 0-padded
   int final_rows;      // 1: every tile is one unit, whose pools are final: the selection
                        // warps write the exact top-K rows themselves (no partial lists)
+  int t0;              // sequence position of query row 0 (0 for a whole prefill)
 };
 
 // A unit leaves at most this many candidates per query (a superset of its K
@@ -517,8 +518,8 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
       if (t >= p.S) continue;
       uint64_t* pool = sm.pool + (size_t)qi * p.cap;
       const long long t_in = role_t0();
-      pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(t, p.T, p.m), pool,
-                      p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane, ctl);
+      pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(p.t0 + t, p.T, p.m),
+                      pool, p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane, ctl);
       if (lane == 0) role_add(ctl, R_SEL_INTAKE, t_in);
       if (md.last) {
         const long long t_end = role_t0();
@@ -571,12 +572,13 @@ struct UnitGrid {
   int tile_units;  // 1: a unit is a whole query tile, its key chunks handled in
                    // order inside it (the tile is loaded once); 0: one unit
                    // per (tile, chunk)
+  int t0;          // sequence position of query row 0, the same in every batch
 };
 
 SI_DEV int tile_vmax(const UnitGrid& u, int g) {
   int t = g * u.QT + u.QT - 1;
   if (t > u.S - 1) t = u.S - 1;
-  return visible_keys(t, u.T, u.m);
+  return visible_keys(u.t0 + t, u.T, u.m);
 }
 
 // Number of chunks of tile g (at least 1, so tiles with no visible key still

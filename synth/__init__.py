@@ -233,6 +233,46 @@ def gen_scores(B: int, S: int, T: int, seed: int = 0, kind: str = "normal") -> n
     raise ValueError(kind)
 
 
+# --------------------------------------------------------------------------- decode
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeShape:
+    """A decode step: the S_q newest queries (positions t0 .. t0+S_q-1) of
+    each of the B sequences described by ``seq``, against the seq.T keys
+    compressed so far.  Its inputs are rows of the sequence's own q and w
+    and the sequence's kc, so a decode step reproduces rows of the prefill
+    workload ``seq``."""
+
+    name: str
+    seq: Shape
+    t0: int
+    S_q: int
+
+    @property
+    def T(self) -> int:
+        return self.seq.T
+
+
+DECODE_SHAPES = {
+    # 64 sequences of 65,536 tokens (16,384 compressed keys each), the next
+    # token of each: the memory-bound regime (268 MB of keys per step)
+    "decode_b64_t16k": DecodeShape(
+        "decode_b64_t16k", Shape("decode_b64_t16k", 64, 65536, 4, 64, 128, 2048, "ar1", 1.0 / 8.0,
+                                 0), 65535, 1),
+}
+
+
+def gen_decode(ds: DecodeShape, seed: int = 0):
+    """(q [B,S_q,H,D] bf16 bits, w [B,S_q,H] fp32, kc [B,T,D] bf16 bits) of a
+    decode step: rows t0 .. t0+S_q-1 of the sequence's q and w, and its kc."""
+    sh = ds.seq
+    rows = (np.arange(sh.B, dtype=np.int64)[:, None] * sh.S
+            + np.minimum(ds.t0 + np.arange(ds.S_q), sh.S - 1)[None, :]).reshape(-1)
+    q, w = gen_rows(sh, rows, seed)
+    return (q.reshape(sh.B, ds.S_q, sh.H, sh.D), w.reshape(sh.B, ds.S_q, sh.H), gen_kc(sh, seed))
+
+
 def small(B: int, S: int, m: int, H: int, D: int, topk: int, seed: int = 0, kc_kind: str = "iid",
           w_scale: float = 0.125) -> Shape:
     """An ad-hoc small workload (tests use these for ragged and edge shapes)."""

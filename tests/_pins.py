@@ -151,7 +151,42 @@ def check_fp8_brute_force(o) -> None:
                 assert abs(got[r, c] - want) <= 1e-14 * max(abs(want), 1e-300), ("fp8 key", r, j)
 
 
+# (seed, B, T, m, H, D, k, t0, S_q): positions that see no key, fewer keys
+# than k, exactly the last key (t0 + i = m*T - 1) and past it (all T keys)
+DECODE = [(31, 2, 4, 3, 2, 3, 3, 0, 4), (32, 2, 4, 3, 2, 3, 3, 9, 6), (33, 1, 5, 2, 3, 2, 4, 8, 5),
+          (34, 3, 3, 1, 2, 2, 2, 1, 4)]
+
+
+def check_decode_brute_force(o) -> None:
+    """The decode oracle (rows, scores, max |score|, key scores through the
+    decode rows) against exact rational arithmetic with each query's own
+    position, on dyadic inputs."""
+    for seed, B, T, m, H, D, k, t0, S_q in DECODE:
+        g = np.random.default_rng(seed)
+        q = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(B, S_q, H, D)).astype(np.float32) / 8)
+        kc = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(B, T, D)).astype(np.float32) / 8)
+        w = (g.integers(-8, 9, size=(B, S_q, H)) / 8).astype(np.float32)
+        bi, bs = brute.topk_decode(q, w, kc, m, k, t0)
+        bsf = np.array([[-np.inf if x is None else float(x) for x in r] for r in bs])
+        oi, os_, am = o.indexer_decode(q, w, kc, t0, m, k)
+        assert np.array_equal(oi, np.array(bi)) and _same_scores(os_, bsf), ("decode", seed)
+        exact = np.full((B * S_q, T), np.nan)
+        for b in range(B):
+            for i in range(S_q):
+                for j in range(brute.visible_count(t0 + i, T, m)):
+                    exact[b * S_q + i, j] = float(brute.score(q, w, kc, b, i, j))
+        assert np.array_equal(am, np.max(np.abs(np.nan_to_num(exact, nan=0.0)), axis=1)), (
+            "decode absmax", seed)
+        S, rows = o.decode_rows(B, S_q, t0, T, m)
+        js = np.broadcast_to(np.arange(-1, T, dtype=np.int32), (B * S_q, T + 1)).copy()
+        got = o.score_keys_rows(q.reshape(B * S_q, H, D), w.reshape(B * S_q, H), kc, S, m, rows,
+                                js)
+        want = np.where(js >= 0, exact[np.arange(B * S_q)[:, None], np.maximum(js, 0)], np.nan)
+        assert np.all((got == want) | (np.isnan(got) & np.isnan(want))), ("decode keys", seed)
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
     check_dyadic_brute_force(o)
     check_fp8_brute_force(o)
+    check_decode_brute_force(o)

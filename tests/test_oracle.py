@@ -186,6 +186,10 @@ def test_pins_fp8_rows_and_key_scores_brute_force():
     _pins.check_fp8_brute_force(oracle)
 
 
+def test_pins_decode_rows_brute_force():
+    _pins.check_decode_brute_force(oracle)
+
+
 def test_row_helpers_match_numpy_two_batches():
     """Random bf16 inputs, two batches, rows t < m - 1 included: the max
     |score| over visible keys and the scores of given keys (visible, -1 and

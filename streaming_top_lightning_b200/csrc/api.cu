@@ -207,17 +207,18 @@ Plan make_plan(int B, int S, int T, int K, int QT, int H, const Opts& o) {
   return p;
 }
 
-// The rows of a query block: from a single candidate list per query (one
-// key chunk) the bucket-sort kernel, else the merge kernel over the chunks.
+// The rows of a query block: the bucket-sort kernel when a query's candidate
+// lists (one per key chunk) hold at most kFinishMaxKeys keys together, else
+// the merge kernel over the chunks.
 cudaError_t finish_launch(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                           cudaStream_t stream) {
-  if (sp.nch_max == 1) return launch_finish_rows(partial, sp, stream);
+  if (finish_takes(sp.L, sp.nch_max)) return launch_finish_rows(partial, sp, ug, stream);
   return launch_merge(partial, sp, ug, stream);
 }
 
 // True when no row-sort pass is needed after the finishing launches.
 bool rows_come_sorted(const Plan& pl, int K) {
-  return rows_sorted_in_warp(K) || (!pl.final_rows && pl.nch_max == 1);
+  return rows_sorted_in_warp(K) || (!pl.final_rows && finish_takes(pl.L, pl.nch_max));
 }
 
 // The selection's invariant: a pool has room for K keys plus one 64-key
@@ -372,7 +373,10 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
   for (int blk = 0; blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, 1, pb.t0};
+    // a prefill's tiles outnumber the SMs: a unit is a whole tile (loaded
+    // once, its chunks in order); a decode step's few tiles are split into
+    // (tile, chunk) units that spread over the SMs
+    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, pb.decode ? 0 : 1, pb.t0};
     ScoreParams p{};
     p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
                       sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,

@@ -1,12 +1,13 @@
-// Exact, sorted top-k rows from one candidate list per query (the case of a
-// single key chunk).
+// Exact, sorted top-k rows from a query's few candidate lists (one per key
+// chunk; a single list when one chunk spans all of the query's keys).
 //
 // "StreamIndex: Memory-Bounded Compressed Sparse Attention via Streaming
 // Top-k", Abstract: the top-k keys are selected per query by a chunked
-// partition-merge driver.  When one chunk spans all of a query's keys, the
-// fused kernel leaves per query one pruned list of at most L candidate keys
-// (a superset of the query's K best, zero-padded); this kernel turns it into
-// the output row.
+// partition-merge driver.  The fused kernel leaves per query and key chunk
+// one pruned list of at most L candidate keys (a superset of that chunk's K
+// best, zero-padded); when a query's lists together hold at most
+// kFinishMaxKeys keys, this kernel turns them into the output row in one
+// pass (longer sets go to the merge kernel).
 //
 // One CTA per query, a bucket (counting) sort instead of a comparison
 // network.  The candidates' 32-bit score images (the high word of the
@@ -72,20 +73,23 @@ struct FinishRed {
   uint32_t n[32], omin[32], omax[32], tot[32], mx[32];
 };
 
-// One CTA per query.  Shared memory: raw[L] (the list as read), tmp[cap]
-// (bucket-ordered candidates), bins[nb] (counts, then bucket starts, then
-// bucket ends), and a small block for cross-warp reductions.
+// One CTA per query.  Shared memory: raw[nl*L] (the query's nl lists as
+// read, one after another), tmp[cap] (bucket-ordered candidates), bins[nb]
+// (counts, then bucket starts, then bucket ends), and a small block for
+// cross-warp reductions.  Only the lists the fused kernel wrote for the
+// query's tile are read: its tile_chunks(), each L keys (L / 2 16-byte words).
 __global__ void __launch_bounds__(256)
-    k_finish_rows(const uint64_t* __restrict__ partial, SelParams sp, int tmp_cap, int nb) {
+    k_finish_rows(const uint64_t* __restrict__ partial, SelParams sp, UnitGrid ug, int raw_cap,
+                  int tmp_cap, int nb) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
   const int nw = nthr >> 5;
-  const int K = sp.K, QT = sp.QT, L = sp.L;
+  const int K = sp.K, QT = sp.QT;
   uint64_t* raw = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* tmp = raw + L;
+  uint64_t* tmp = raw + raw_cap;
   uint32_t* bins = reinterpret_cast<uint32_t*>(tmp + tmp_cap);
   uint16_t* rawb = reinterpret_cast<uint16_t*>(bins + nb);  // bucket of raw[i]
-  uint16_t* tmpb = rawb + L;                                // bucket of tmp[i]
+  uint16_t* tmpb = rawb + raw_cap;                          // bucket of tmp[i]
   FinishRed* red = reinterpret_cast<FinishRed*>(tmpb + tmp_cap);
   const uint32_t qid = blockIdx.x;  // < B*S < 2^31
   const uint32_t tq = qid / (uint32_t)QT;
@@ -94,16 +98,22 @@ __global__ void __launch_bounds__(256)
   const int gl = (int)(tq - (uint32_t)b * (uint32_t)sp.n_tiles);
   const int t = (sp.g_lo + gl) * QT + qi;
   if (t >= sp.S) return;
-  const uint64_t* src = partial + (((int64_t)b * sp.n_tiles + gl) * sp.nch_max * QT + qi) * L;
+  const int nl = sp.nch_max == 1 ? 1 : min(tile_chunks(ug, sp.g_lo + gl), sp.nch_max);
+  const int L = nl * sp.L;  // candidates read (nl lists), at most raw_cap
+  if (L > raw_cap) return;  // the host sizes raw_cap for every tile; never taken
+  // list c of the query: partial[b][gl][c][qi][0 .. sp.L)
+  const uint64_t* src = partial + (((int64_t)b * sp.n_tiles + gl) * sp.nch_max * QT + qi) * sp.L;
+  const int64_t list_stride4 = (int64_t)QT * sp.L / 2;  // 16-byte words between lists
+  const int l4 = sp.L / 2;                                // 16-byte words of one list
   int32_t* oi = sp.out_idx + ((int64_t)b * sp.S + t) * K;
   float* os = sp.out_score + ((int64_t)b * sp.S + t) * K;
 
-  // pass 1: the list into shared memory (16-byte loads, all issued before any
-  // is used), the count of real candidates (non-zero keys) and the range of
-  // their score images
+  // pass 1: the lists into shared memory (16-byte loads, all issued before
+  // any is used), the count of real candidates (non-zero keys) and the range
+  // of their score images
   uint32_t n = 0, omin = 0xFFFFFFFFu, omax = 0u;
   {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src);  // L is a multiple of 32
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);  // sp.L is a multiple of 32
     uint4* r4 = reinterpret_cast<uint4*>(raw);
     const int n4 = L / 2;
     for (int i0 = 0; i0 < n4; i0 += 4 * nthr) {
@@ -111,7 +121,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u * nthr + tid;
-        v[u] = i < n4 ? __ldg(s4 + i) : make_uint4(0u, 0u, 0u, 0u);
+        const int c = i / l4;
+        v[u] = i < n4 ? __ldg(s4 + c * list_stride4 + (i - c * l4)) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -277,33 +288,38 @@ __global__ void __launch_bounds__(256)
 }
 
 // Launch shape: a CTA per query, 128 threads for short lists and 256 for
-// long ones; buckets: twice the list length rounded up to a power of two,
-// within [1024, 8192], so that the crowded buckets near the K-th score stay
-// short; room for the gathered candidates:
-// the whole list, and a power of two at least K for the fallback sort.
+// long ones; buckets: twice the candidate count rounded up to a power of
+// two, within [1024, 8192], so that the crowded buckets near the K-th score
+// stay short; room for the gathered candidates: all of them, and a power of
+// two at least K for the fallback sort.
 struct FinishShape {
-  int threads, nb, tmp_cap;
+  int threads, nb, raw_cap, tmp_cap;
   size_t smem;
 };
 
-static FinishShape finish_shape(int K, int L) {
+static FinishShape finish_shape(int K, int L, int nch) {
   FinishShape f;
-  f.threads = L > 1024 ? 256 : 128;
-  f.nb = std::min(8192, std::max(1024, 2 * (int)pow2ceil(L)));
-  f.tmp_cap = std::max(L, (int)pow2ceil(K));
-  f.smem = (sizeof(uint64_t) + sizeof(uint16_t)) * ((size_t)L + f.tmp_cap) +
+  f.raw_cap = L * nch;
+  f.threads = f.raw_cap > 1024 ? 256 : 128;
+  f.nb = std::min(8192, std::max(1024, 2 * (int)pow2ceil(f.raw_cap)));
+  f.tmp_cap = std::max(f.raw_cap, (int)pow2ceil(K));
+  f.smem = (sizeof(uint64_t) + sizeof(uint16_t)) * ((size_t)f.raw_cap + f.tmp_cap) +
            sizeof(uint32_t) * f.nb + sizeof(FinishRed) + 16;
   return f;
 }
 
-cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp,
+bool finish_takes(int L, int nch) { return (int64_t)L * nch <= kFinishMaxKeys; }
+
+cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                                cudaStream_t stream) {
-  const FinishShape f = finish_shape(sp.K, sp.L);
+  if (!finish_takes(sp.L, sp.nch_max)) return cudaErrorInvalidValue;
+  const FinishShape f = finish_shape(sp.K, sp.L, sp.nch_max);
   cudaError_t e = cudaFuncSetAttribute(k_finish_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)f.smem);
   if (e != cudaSuccess) return e;
   const int64_t queries = (int64_t)sp.B * sp.n_tiles * sp.QT;
-  k_finish_rows<<<(unsigned)queries, f.threads, f.smem, stream>>>(partial, sp, f.tmp_cap, f.nb);
+  k_finish_rows<<<(unsigned)queries, f.threads, f.smem, stream>>>(partial, sp, ug, f.raw_cap,
+                                                                   f.tmp_cap, f.nb);
   return cudaGetLastError();
 }
 

@@ -64,7 +64,13 @@ bool merge_sorts_rows(int K);
 
 // Exact sorted rows from a single candidate list per query (one key chunk);
 // every row comes out sorted, whatever K.
-cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, cudaStream_t stream);
+// The finishing kernel takes a query's lists when they hold at most this many
+// keys together (its shared memory, and the fallback select's byte counters:
+// at most 255 * 32 keys); longer sets go through the merge kernel.
+constexpr int kFinishMaxKeys = 8160;
+bool finish_takes(int L, int nch);
+cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
+                               cudaStream_t stream);
 
 // Sorts each of the rows [rows, K] of (idx, score) in place into the output
 // order (score descending, index ascending, padding last).

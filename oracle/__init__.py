@@ -69,6 +69,9 @@ def declare(lib):
     lib.oracle_indexer_topk_fp8_rows.restype = I
     lib.oracle_score_keys_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, I, P]
     lib.oracle_score_keys_fp8_rows.restype = None
+    lib.oracle_sparse_attention_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double,
+                                                 P, P]
+    lib.oracle_sparse_attention_rows.restype = I
     return lib
 
 
@@ -218,6 +221,26 @@ def indexer_decode(q, w, kc, t0: int, m: int, k: int, lib=None):
                                     rows, lib=lib)
 
 
+def sparse_attention_rows(qa_rows, ka, va, idx_rows, batch, scale: float, lib=None):
+    """Multi-query attention of each listed query row over its listed entries
+    (see oracle_sparse_attention_rows): qa_rows [n,H,D] bf16 bits, ka and va
+    [B,T,D] bf16 bits, idx_rows [n,k] int32, batch [n] (each row's batch).
+    Returns (out [n,H,D], absw [n,H,D]) in fp64."""
+    qa_rows, ka, va = _c(qa_rows, np.uint16), _c(ka, np.uint16), _c(va, np.uint16)
+    idx_rows, batch = _c(idx_rows, np.int32), _c(batch, np.int64)
+    n, H, D = qa_rows.shape
+    B, T = ka.shape[0], ka.shape[1]
+    k = idx_rows.shape[1]
+    out = np.empty((n, H, D), dtype=np.float64)
+    absw = np.empty((n, H, D), dtype=np.float64)
+    rc = _use(lib).oracle_sparse_attention_rows(_p(qa_rows), _p(ka), _p(va), _p(idx_rows),
+                                                _p(batch), n, B, T, H, D, k, float(scale),
+                                                _p(out), _p(absw))
+    if rc != 0:
+        raise ValueError("oracle_sparse_attention_rows: bad arguments")
+    return out, absw
+
+
 def topk_scores(X, m: int, k: int, rows=None, lib=None):
     """Selection alone on given fp32 scores X [B,S,T].
     Returns (idx [n,k] int32, score [n,k] float32 carrying the input bit patterns)."""
@@ -289,4 +312,4 @@ _API = {name: globals()[name] for name in (
     "threads", "visible", "indexer_topk", "indexer_topk_rows", "indexer_topk_rows_absmax",
     "score_keys_rows", "row_absmax_rows", "topk_scores", "e4m3_decode", "e4m3_encode",
     "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows", "decode_rows",
-    "indexer_decode")}
+    "indexer_decode", "sparse_attention_rows")}

@@ -420,3 +420,77 @@ void oracle_score_keys_fp8_rows(const uint8_t* q8_rows, const float* sq_rows, co
         }
     }
 }
+
+/* ------------------------------------------------------------ sparse attention
+ * The consumer of the indexer's rows ("StreamIndex: Memory-Bounded Compressed
+ * Sparse Attention via Streaming Top-k", Abstract: the top-k keys are kept per
+ * query and a sparse attention kernel reads only those).  The abstract gives
+ * no formula; the reading used here is multi-query attention over the listed
+ * compressed entries, every query head sharing one key row and one value row
+ * per entry:
+ *
+ *   J = the listed entries idx[r], 0 <= r < k, with 0 <= idx[r] < T
+ *       (padding -1 and out-of-range entries skipped; entries count as listed)
+ *   l_j(h) = scale * sum_d qa[h,d] * ka[j,d]
+ *   o[h,:] = sum_{j in J} exp(l_j(h) - M) * va[j,:] / sum_{j in J} exp(l_j(h) - M),
+ *            M = max_{j in J} l_j(h)                (o = 0 when J is empty)
+ *
+ * and, for the tolerance of a lower-precision result, the probability-
+ * weighted magnitude a[h,d] = sum_j p_j(h) * |va[j,d]|.  fp64 throughout, sums
+ * in ascending d and in list order.
+ *
+ * qa_rows [n,H,D] bf16 (row i belongs to batch batch[i]); ka, va [B,T,D]
+ * bf16; idx_rows [n,k]; out, absw [n,H,D].  Returns -1 on bad sizes.
+ */
+int oracle_sparse_attention_rows(const uint16_t* qa_rows, const uint16_t* ka, const uint16_t* va,
+                                 const int32_t* idx_rows, const int64_t* batch, int n, int B,
+                                 int T, int H, int D, int k, double scale, double* out,
+                                 double* absw) {
+    if (n < 0 || B < 1 || T < 1 || H < 1 || D < 1 || k < 1) return -1;
+    for (int i = 0; i < n; i++)
+        if (batch[i] < 0 || batch[i] >= B) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n; i++) {
+        const int32_t* ir = idx_rows + (int64_t)i * k;
+        const uint16_t* kb = ka + batch[i] * (int64_t)T * D;
+        const uint16_t* vb = va + batch[i] * (int64_t)T * D;
+        double* l = (double*)malloc(sizeof(double) * (size_t)k);
+        for (int h = 0; h < H; h++) {
+            const uint16_t* qh = qa_rows + ((int64_t)i * H + h) * D;
+            double* oh = out + ((int64_t)i * H + h) * D;
+            double* ah = absw + ((int64_t)i * H + h) * D;
+            for (int d = 0; d < D; d++) oh[d] = ah[d] = 0.0;
+            double M = -INFINITY;
+            int any = 0;
+            for (int r = 0; r < k; r++) {
+                const int j = ir[r];
+                if (j < 0 || j >= T) continue;
+                double s = 0.0;
+                for (int d = 0; d < D; d++)
+                    s += bf16_to_f64(qh[d]) * bf16_to_f64(kb[(int64_t)j * D + d]);
+                l[r] = scale * s;
+                if (!any || l[r] > M) M = l[r];
+                any = 1;
+            }
+            if (!any) continue;
+            double Z = 0.0;
+            for (int r = 0; r < k; r++) {
+                const int j = ir[r];
+                if (j < 0 || j >= T) continue;
+                Z += exp(l[r] - M);
+            }
+            for (int r = 0; r < k; r++) {
+                const int j = ir[r];
+                if (j < 0 || j >= T) continue;
+                const double p = exp(l[r] - M) / Z;
+                for (int d = 0; d < D; d++) {
+                    const double v = bf16_to_f64(vb[(int64_t)j * D + d]);
+                    oh[d] += p * v;
+                    ah[d] += p * fabs(v);
+                }
+            }
+        }
+        free(l);
+    }
+    return 0;
+}

@@ -185,8 +185,82 @@ def check_decode_brute_force(o) -> None:
         assert np.all((got == want) | (np.isnan(got) & np.isnan(want))), ("decode keys", seed)
 
 
+def _sdpa_rows(qa, ka, va, idx, batch, scale):
+    """The same attention through a library routine: torch's scaled dot-product
+    attention in fp64 on the CPU, with a boolean mask over all T entries
+    selecting the listed ones (rows with no listed entry give 0)."""
+    import torch
+
+    n, H, D = qa.shape
+    T = ka.shape[1]
+    out = np.zeros((n, H, D))
+    for i in range(n):
+        sel = idx[i][(idx[i] >= 0) & (idx[i] < T)]
+        if sel.size == 0:
+            continue
+        mask = torch.zeros((1, 1, 1, T), dtype=torch.bool)
+        mask[..., torch.from_numpy(sel.astype(np.int64))] = True
+        q = torch.from_numpy(synth.bf16_bits_to_f32(qa[i]).astype(np.float64))[None, :, None, :]
+        kk = torch.from_numpy(synth.bf16_bits_to_f32(ka[batch[i]]).astype(np.float64))
+        vv = torch.from_numpy(synth.bf16_bits_to_f32(va[batch[i]]).astype(np.float64))
+        kk = kk[None, None].expand(1, H, T, D)
+        vv = vv[None, None].expand(1, H, T, D)
+        o = torch.nn.functional.scaled_dot_product_attention(q, kk, vv, attn_mask=mask,
+                                                             scale=scale)
+        out[i] = o[0, :, 0, :].numpy()
+    return out
+
+
+def check_sparse_attention(o) -> None:
+    """The attention oracle against (a) torch's fp64 scaled dot-product
+    attention with a mask of the listed entries, on random rows with padding,
+    out-of-range entries and two batches; (b) closed forms: one listed entry
+    gives its value row exactly, all-equal logits give the mean of the listed
+    value rows, two entries whose logits differ by ln 3 get weights 1/4 and
+    3/4; (c) the weighted magnitude equals the output when every value is
+    non-negative, and is 0 with the output for a row with no entry."""
+    g = np.random.default_rng(41)
+    B, T, H, D, k, n = 2, 9, 3, 4, 5, 7
+    qa = synth.f32_to_bf16_bits(g.standard_normal((n, H, D)).astype(np.float32))
+    ka = synth.f32_to_bf16_bits(g.standard_normal((B, T, D)).astype(np.float32))
+    va = synth.f32_to_bf16_bits(g.standard_normal((B, T, D)).astype(np.float32))
+    idx = np.stack([g.permutation(T)[:k] for _ in range(n)]).astype(np.int32)
+    idx[1, 3:] = -1          # padding
+    idx[2, 0] = T            # out of range: skipped
+    idx[3, :] = -1           # no entry
+    batch = np.array([0, 1, 1, 0, 1, 0, 1], dtype=np.int64)
+    scale = 0.37
+    out, absw = o.sparse_attention_rows(qa, ka, va, idx, batch, scale)
+    ref = _sdpa_rows(qa, ka, va, idx, batch, scale)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-13), ("sparse attention vs sdpa", out, ref)
+    assert np.all(out[3] == 0) and np.all(absw[3] == 0), "row with no entry"
+    # closed forms, on dyadic values
+    one = lambda x: synth.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))  # noqa: E731
+    ka1 = one([[[1, 0], [0, 1], [0.5, 0.5], [1, 1]]])                          # [1, 4, 2]
+    va1 = one([[[2, -3], [0.25, 4], [-1, 1], [8, 0.5]]])
+    qa1 = one([[[1, 0], [0, 0]]])                                             # head 1: q = 0
+    out1, _ = o.sparse_attention_rows(qa1, ka1, va1, np.array([[2, -1, -1]], np.int32),
+                                      np.array([0]), 1.0)
+    assert np.array_equal(out1[0, 0], [-1.0, 1.0]) and np.array_equal(out1[0, 1], [-1.0, 1.0])
+    out2, _ = o.sparse_attention_rows(qa1, ka1, va1, np.array([[0, 1, 3]], np.int32),
+                                      np.array([0]), 1.0)
+    assert np.allclose(out2[0, 1], (np.array([2, -3]) + [0.25, 4] + [8, 0.5]) / 3, rtol=1e-15)
+    out3, _ = o.sparse_attention_rows(qa1, ka1, va1, np.array([[1, 0]], np.int32), np.array([0]),
+                                      float(np.log(3.0)))
+    # head 0: logits 0 (entry 1) and ln 3 (entry 0): weights 1/4 and 3/4
+    assert np.allclose(out3[0, 0], 0.25 * np.array([0.25, 4]) + 0.75 * np.array([2, -3]),
+                       rtol=1e-14, atol=1e-15)
+    vpos = one(np.abs(g.standard_normal((B, T, D))))
+    outp, absp = o.sparse_attention_rows(qa, ka, vpos, idx, batch, scale)
+    assert np.allclose(outp, absp, rtol=1e-14, atol=0), "weighted magnitude, non-negative values"
+    # the weighted magnitude is the attention output of |v| (library route)
+    vabs = one(np.abs(synth.bf16_bits_to_f32(va)))
+    assert np.allclose(absw, _sdpa_rows(qa, ka, vabs, idx, batch, scale), rtol=1e-12, atol=1e-13)
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
     check_dyadic_brute_force(o)
     check_fp8_brute_force(o)
     check_decode_brute_force(o)
+    check_sparse_attention(o)

@@ -81,6 +81,17 @@ MUTATIONS = {
                                      "            out[(int64_t)i * kk + r] = oracle_score_row_fp8(",
                                      "            if (j < 0) continue;\n"
                                      "            out[(int64_t)i * kk + r] = oracle_score_row_fp8("),
+    # sparse attention over the listed entries
+    "attn_scale_dropped": ("                l[r] = scale * s;", "                l[r] = s;"),
+    "attn_query_of_head_0": ("            const uint16_t* qh = qa_rows + ((int64_t)i * H + h) * D;",
+                             "            const uint16_t* qh = qa_rows + ((int64_t)i * H) * D;"),
+    "attn_no_batch_offset": ("        const uint16_t* vb = va + batch[i] * (int64_t)T * D;",
+                             "        const uint16_t* vb = va;"),
+    "attn_value_of_first_entry": ("                    const double v = bf16_to_f64(vb[(int64_t)j * D + d]);",
+                                  "                    const double v = bf16_to_f64(vb[(int64_t)ir[0] * D + d]);"),
+    "attn_normaliser_skips_first": ("            double Z = 0.0;\n            for (int r = 0; r < k; r++) {",
+                                    "            double Z = 0.0;\n            for (int r = 1; r < k; r++) {"),
+    "attn_absw_without_abs": ("                    ah[d] += p * fabs(v);", "                    ah[d] += p * v;"),
 }
 
 

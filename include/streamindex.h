@@ -275,6 +275,32 @@ int si_indexer_decode_workspace_size(int B, int S_q, int t0, int T, int H_I, int
 int si_indexer_decode_plan(int B, int S_q, int t0, int T, int H_I, int d_I, int m, int topk,
                            const si_options* opt, si_plan_info* out);
 
+/* ---- sparse attention over the selected entries -------------------------- */
+
+/*
+ * si_sparse_attention: the consumer of the indexer's rows.  The abstract
+ * describes it only as a sparse attention kernel that reads the selected
+ * keys; this call computes multi-query attention over the entries a row
+ * lists, all query heads sharing one key row and one value row per entry:
+ *   J(b,t) = { idx[b,t,r] : 0 <= r < topk, 0 <= idx[b,t,r] < T }
+ *   out[b,t,h,:] = sum_{j in J} softmax_j(scale * qa[b,t,h,:] . ka[b,j,:]) * va[b,j,:]
+ * (entries count as listed; -1 padding and out-of-range entries are skipped;
+ * a row that lists none gives zeros).
+ *   qa   bf16 [B,S,H_a,d_a]   query heads (H_a = 128, d_a = 128)
+ *   ka   bf16 [B,T,d_a]       key rows of the compressed entries
+ *   va   bf16 [B,T,d_a]       value rows
+ *   idx  int32 [B,S,topk]     the entries of each query (si_indexer_topk's out_idx)
+ *   out  fp32 [B,S,H_a,d_a]
+ * Arithmetic: q.k in fp32 from bf16 products on the tensor cores, softmax
+ * in fp32, the probabilities rounded to bf16 for the weighted sum of the
+ * value rows (accumulated in fp32).  Limits: 1 <= topk <= 2048; B*S*H_a <
+ * 2^31; qa, ka, va, out 16-byte aligned, idx 4-byte aligned; scale finite.
+ * Options: grid_ctas and timeout_ms are used.  No workspace.
+ */
+int si_sparse_attention(const void* qa, const void* ka, const void* va, const int32_t* idx, int B,
+                        int S, int T, int H_a, int d_a, int topk, float scale, float* out,
+                        const si_options* opt, void* stream);
+
 /* ---- diagnostics ------------------------------------------------------ */
 
 /* Text for a status code (static storage). */

@@ -196,6 +196,33 @@ def indexer_decode(q, w, kc, t0: int, m: int, topk: int, *, out=None,
     return idx, score
 
 
+def sparse_attention(qa, ka, va, idx, scale: float | None = None, *, out=None,
+                     opts: SiOptions | None = None, stream=None):
+    """Multi-query attention of each query's heads over the entries its row of
+    ``idx`` lists (si_sparse_attention): qa [B,S,128,128] bf16, ka and va
+    [B,T,128] bf16, idx [B,S,topk] int32 (-1 padding).  ``scale`` defaults to
+    1/sqrt(128).  Returns out [B,S,128,128] fp32."""
+    torch = _torch()
+    _need(qa, torch.bfloat16, 4, "qa")
+    _need(ka, torch.bfloat16, 3, "ka")
+    _need(va, torch.bfloat16, 3, "va")
+    _need(idx, torch.int32, 3, "idx")
+    B, S, H, D = qa.shape
+    T = ka.shape[1]
+    if tuple(va.shape) != tuple(ka.shape) or idx.shape[0] != B or idx.shape[1] != S:
+        raise ValueError("ka, va must be [B,T,D] and idx [B,S,topk]")
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty((B, S, H, D), dtype=torch.float32, device=qa.device)
+    _need(out, torch.float32, 4, "out")
+    rc = _lib.load().si_sparse_attention(_ptr(qa), _ptr(ka), _ptr(va), _ptr(idx), B, S, T, H, D,
+                                         idx.shape[2], float(scale), _ptr(out),
+                                         ctypes.byref(opts) if opts else None, _stream(stream))
+    _lib.check("si_sparse_attention", rc)
+    return out
+
+
 def indexer_topk_noalloc(q, w, kc, m: int, topk: int, *, out=None, stream=None):
     """``indexer_topk`` through the entry point that allocates no device memory
     (its scratch is a fixed array inside the library; see

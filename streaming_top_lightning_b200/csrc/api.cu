@@ -710,6 +710,48 @@ int si_indexer_topk_noalloc(const void* q, const float* w, const void* kc, int B
                      out_score, &opt, ws, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------ sparse attention
+int si_sparse_attention(const void* qa, const void* ka, const void* va, const int32_t* idx, int B,
+                        int S, int T, int H_a, int d_a, int topk, float scale, float* out,
+                        const si_options* opt, void* stream) {
+  if (!qa || !ka || !va || !idx || !out) return SI_ERR_NULL;
+  if (B < 1 || S < 1 || T < 1 || H_a != 128 || d_a != 128) return SI_ERR_DIM;
+  if ((int64_t)B * S * H_a >= ((int64_t)1 << 31)) return SI_ERR_DIM;
+  if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
+  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return SI_ERR_OPTIONS;
+  if (!aligned16(qa) || !aligned16(ka) || !aligned16(va) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return SI_ERR_ALIGN;
+  Opts o;
+  int rc = read_opts(opt, &o);
+  if (rc) return rc;
+  DevInfo* dev;
+  if ((rc = dev_info(&dev))) return rc;
+  if (sparse_attn_smem_bytes() > (size_t)dev->max_smem) return SI_ERR_UNSUPPORTED;
+  CUtensorMap tm_q;
+  if ((rc = make_map(&tm_q, qa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)B * S * H_a, d_a, 2,
+                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+    return rc;
+  AttnParams p{};
+  p.ka = static_cast<const uint16_t*>(ka);
+  p.va = static_cast<const uint16_t*>(va);
+  p.idx = idx;
+  p.out = out;
+  p.B = B;
+  p.S = S;
+  p.T = T;
+  p.k = topk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = dev->err;
+  p.timeout_ns = (uint64_t)o.timeout_ms * 1000000ull;
+  const int64_t queries = (int64_t)B * S;
+  int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
+  if (grid > queries) grid = (int)queries;
+  return launch_sparse_attn(tm_q, p, grid, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SI_OK
+             : SI_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ decode
 int si_indexer_decode_workspace_size(int B, int S_q, int t0, int T, int H_I, int d_I, int m,
                                      int topk, const si_options* opt, size_t* bytes) {

@@ -27,6 +27,21 @@ struct ScoreParams {
   unsigned long long* role;  // role counters of a profiling build, else null
 };
 
+// Parameters of the sparse attention kernel (128 heads of dim 128).
+struct AttnParams {
+  const uint16_t* ka;  // [B*T, 128] bf16 key rows
+  const uint16_t* va;  // [B*T, 128] bf16 value rows
+  const int32_t* idx;  // [B*S, k] listed entries (-1: none)
+  float* out;          // [B*S, 128, 128] fp32
+  int B, S, T, k;
+  float scale_log2;    // softmax scale times log2(e)
+  uint32_t* err;       // device error word
+  uint64_t timeout_ns; // limit of any single wait
+};
+size_t sparse_attn_smem_bytes();
+cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const AttnParams& p, int grid,
+                               cudaStream_t stream);
+
 // Shared-memory plan of the fused kernel for one problem shape.
 struct ScorePlan {
   int QT;        // queries per tile (nq / H)

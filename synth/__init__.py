@@ -273,6 +273,21 @@ def gen_decode(ds: DecodeShape, seed: int = 0):
     return (q.reshape(sh.B, ds.S_q, sh.H, sh.D), w.reshape(sh.B, ds.S_q, sh.H), gen_kc(sh, seed))
 
 
+# --------------------------------------------------------------------------- attention
+
+
+def gen_attention(B: int, S: int, T: int, H: int = 128, D: int = 128, seed: int = 0):
+    """Inputs of the sparse attention over the selected entries: query heads
+    qa [B,S,H,D] and the entries' key and value rows ka, va [B,T,D], all iid
+    N(0,1) rounded to bf16 bits (the softmax scale 1/sqrt(D) then gives
+    logits of unit spread)."""
+    g = _rng(seed, 16, B, S, T)
+    qa = f32_to_bf16_bits(g.standard_normal((B, S, H, D), dtype=np.float32))
+    ka = f32_to_bf16_bits(g.standard_normal((B, T, D), dtype=np.float32))
+    va = f32_to_bf16_bits(g.standard_normal((B, T, D), dtype=np.float32))
+    return qa, ka, va
+
+
 def small(B: int, S: int, m: int, H: int, D: int, topk: int, seed: int = 0, kc_kind: str = "iid",
           w_scale: float = 0.125) -> Shape:
     """An ad-hoc small workload (tests use these for ragged and edge shapes)."""

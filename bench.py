@@ -39,6 +39,7 @@ import synth  # noqa: E402
 
 METRIC = "indexer query-key pairs/sec, TFLOPS vs B200 peak, peak HBM GB at 1 GPU"
 METRIC_DECODE = "decode indexer query-key pairs/sec, HBM GB/s vs B200 peak"
+METRIC_LAYER = "sparse attention query-entry pairs/sec, TFLOPS vs B200 peak, indexer share of the layer"
 UNIT = "pairs/s"
 KERNEL_SRC = os.path.join(ROOT, "streaming_top_lightning_b200", "csrc", "k_score_topk.cu")
 
@@ -712,6 +713,98 @@ def run_decode(args, ds):
     return 0
 
 
+# --------------------------------------------------------------------------- layer
+
+
+def run_layer(args, name):
+    """A compressed-sparse-attention layer: the indexer step, then multi-query
+    attention of 128 heads (dim 128) over the entries it selects.  Times the
+    attention kernel alone (CUDA events around its launch) and the whole
+    layer; the attention's bound is the tensor cores (4 * 128 * 128 flops per
+    query-entry pair: Q K^T and P V)."""
+    import torch
+
+    import streaming_top_lightning_b200 as stl
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("layer workloads run on one GPU")
+    sh = synth.shape(synth.ATTENTION_LAYERS[name])
+    dev = torch.device("cuda", 0)
+    q, w, kc = (synth.gen_q(sh, 0, threads=16), synth.gen_w(sh, 0), synth.gen_kc(sh, 0))
+    qa, ka, va = synth.gen_attention(sh.B, sh.S, sh.T, seed=1)
+    to_bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    q_d, kc_d, qa_d, ka_d, va_d = to_bf(q), to_bf(kc), to_bf(qa), to_bf(ka), to_bf(va)
+    w_d = torch.from_numpy(w).to(dev)
+    del q, qa
+    idx = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32, device=dev)
+    score = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32, device=dev)
+    out = torch.empty((sh.B, sh.S, 128, 128), dtype=torch.float32, device=dev)
+    opts = stl.options()
+    ws = torch.empty(max(16, stl.workspace_size(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, opts)),
+                     dtype=torch.uint8, device=dev)
+    scale = 1.0 / np.sqrt(128.0)
+    stream = torch.cuda.current_stream()
+
+    def indexer():
+        stl.indexer_topk(q_d, w_d, kc_d, sh.m, sh.topk, out=(idx, score), opts=opts, workspace=ws)
+
+    def attention():
+        stl.sparse_attention(qa_d, ka_d, va_d, idx, scale, out=out)
+
+    for _ in range(max(3, args.warmup)):
+        indexer()
+        attention()
+    torch.cuda.synchronize()
+    if stl.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    pairs = int((idx >= 0).sum().item())  # listed entries, as the indexer selected them
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        pass
+    with ClockSampler(uuid) as clk:
+        torch.cuda.synchronize()
+        for i in range(K):
+            ev[i][0].record(stream)
+            indexer()
+            ev[i][1].record(stream)
+            attention()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if stl.device_error() != 0:
+        raise RuntimeError("device error in the timed region")
+    idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    flops = pairs * 4 * 128 * 128
+    peaks, peak_src = measured_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC_LAYER, "value": pairs / (attn_ms / 1e3), "unit": "pairs/s",
+        "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": idx_ms + attn_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; the indexer's own rows select the entries)",
+        "config": {"workload": name, "indexer": sh.name, "B": sh.B, "S": sh.S, "T": sh.T,
+                   "topk": sh.topk, "H_a": 128, "d_a": 128, "listed_pairs": pairs,
+                   "l2": "inputs larger than L2 (query heads)"},
+        "indexer_ms": idx_ms, "attention_ms": attn_ms,
+        "indexer_share_of_layer": idx_ms / (idx_ms + attn_ms),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "traffic": None, "kernel": "k_sparse_attn",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "algorithmic_flops_per_step": flops,
+                     "timing": "CUDA events around the attention launch"},
+        "gpu_launches": K * (stl.plan(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk)["launches"] + 1),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -719,7 +812,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="long_s256k",
-                    choices=sorted(synth.SHAPES) + sorted(synth.DECODE_SHAPES))
+                    choices=sorted(synth.SHAPES) + sorted(synth.DECODE_SHAPES)
+                    + sorted(synth.ATTENTION_LAYERS))
     ap.add_argument("--key-chunk", type=int, default=0)
     ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
                     help="1: rows finished in the fused kernel; 2: by the merge kernel; "
@@ -734,6 +828,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
+    if args.workload in synth.ATTENTION_LAYERS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "layer workloads time the GPU "
+                              "path only; the oracle's attention is timed in the tests"}))
+            return 0
+        return run_layer(args, args.workload)
     if args.workload in synth.DECODE_SHAPES:
         ds = synth.DECODE_SHAPES[args.workload]
         if args.fp8 or args.topk or args.key_tile or args.strip_slots or args.row_finish:

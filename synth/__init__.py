@@ -276,6 +276,14 @@ def gen_decode(ds: DecodeShape, seed: int = 0):
 # --------------------------------------------------------------------------- attention
 
 
+# A layer: the indexer step of SHAPES[indexer] followed by the attention of
+# 128 heads of dim 128 over the entries it selects.
+ATTENTION_LAYERS = {
+    "layer_s16k": "v4flash_s16k",     # S = 16,384, top-512
+    "layer_s64k": "large_s64k",       # S = 65,536, top-2048
+}
+
+
 def gen_attention(B: int, S: int, T: int, H: int = 128, D: int = 128, seed: int = 0):
     """Inputs of the sparse attention over the selected entries: query heads
     qa [B,S,H,D] and the entries' key and value rows ka, va [B,T,D], all iid

@@ -241,6 +241,45 @@ def sparse_attention_rows(qa_rows, ka, va, idx_rows, batch, scale: float, lib=No
     return out, absw
 
 
+def pivot_rows(q, w, kc, m: int, k: int, G: int, C: int, rows, lib=None):
+    """Query-group candidate scan (the PIVOT news page: nearby queries share one
+    prefix scan).  Reading used: the queries of a batch form groups of G
+    consecutive positions; the group's last position (which sees the most keys)
+    scans its visible keys once and keeps its C best by the exact score
+    (score descending, index ascending); each query of the group then ranks
+    only those candidates it can see, by its own exact score, and keeps its k
+    best (padding -1 / -inf).
+
+    q [B,S,H,D] bf16 bits, w [B,S,H], kc [B,T,D]; rows: flat rows b*S + t to
+    evaluate.  Returns (idx [n,k], score [n,k] fp64, absmax [n]: the largest
+    |score| over the row's visible candidates)."""
+    q, w, kc = _c(q, np.uint16), _c(w, np.float32), _c(kc, np.uint16)
+    B, S, H, D = q.shape
+    T = kc.shape[1]
+    rows = np.asarray(rows, dtype=np.int64)
+    reps = np.unique((rows // S) * S + np.minimum((rows % S) // G * G + G - 1, S - 1))
+    qf, wf = q.reshape(B * S, H, D), w.reshape(B * S, H)
+    rep_idx, _ = indexer_topk_rows(qf[reps], wf[reps], kc, S, m, C, reps, lib=lib)
+    cand = {int(r): c[c >= 0] for r, c in zip(reps, rep_idx)}
+    out_i = np.full((rows.size, k), -1, dtype=np.int32)
+    out_s = np.full((rows.size, k), -np.inf)
+    amax = np.zeros(rows.size)
+    for n, r in enumerate(rows):
+        b, t = divmod(int(r), S)
+        rep = b * S + min(t // G * G + G - 1, S - 1)
+        V = min(T, (t + 1) // m)
+        js = np.sort(cand[rep][cand[rep] < V]).astype(np.int32)
+        if js.size == 0:
+            continue
+        sc = score_keys_rows(qf[r:r + 1], wf[r:r + 1], kc, S, m, np.array([r]), js[None, :],
+                             lib=lib)[0]
+        order = np.lexsort((js, -sc))[:k]
+        out_i[n, :order.size] = js[order]
+        out_s[n, :order.size] = sc[order]
+        amax[n] = np.max(np.abs(sc))
+    return out_i, out_s, amax
+
+
 def topk_scores(X, m: int, k: int, rows=None, lib=None):
     """Selection alone on given fp32 scores X [B,S,T].
     Returns (idx [n,k] int32, score [n,k] float32 carrying the input bit patterns)."""
@@ -312,4 +351,4 @@ _API = {name: globals()[name] for name in (
     "threads", "visible", "indexer_topk", "indexer_topk_rows", "indexer_topk_rows_absmax",
     "score_keys_rows", "row_absmax_rows", "topk_scores", "e4m3_decode", "e4m3_encode",
     "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows", "decode_rows",
-    "indexer_decode", "sparse_attention_rows")}
+    "indexer_decode", "sparse_attention_rows", "pivot_rows")}

@@ -76,6 +76,31 @@ def topk_decode(q, w, kc, m: int, k: int, t0: int):
     return out_idx, out_sc
 
 
+def topk_pivot(q, w, kc, m: int, k: int, G: int, C: int):
+    """Query-group candidate scan in exact arithmetic: the last position of
+    each group of G keeps its C best visible keys; every query of the group
+    ranks the candidates it can see by its own score and keeps k."""
+    B, S = q.shape[0], q.shape[1]
+    T = kc.shape[1]
+    out_idx, out_sc = [], []
+    for b in range(B):
+        cand = {}
+        for t in range(S):
+            rep = min(t // G * G + G - 1, S - 1)
+            if rep not in cand:
+                Vr = visible_count(rep, T, m)
+                pr = sorted(((score(q, w, kc, b, rep, j), j) for j in range(Vr)),
+                            key=lambda p: (-p[0], p[1]))
+                cand[rep] = [j for _, j in pr[:C]]
+            V = visible_count(t, T, m)
+            pairs = [(score(q, w, kc, b, t, j), j) for j in cand[rep] if j < V]
+            pairs.sort(key=lambda p: (-p[0], p[1]))
+            sel = pairs[:k]
+            out_idx.append([j for _, j in sel] + [-1] * (k - len(sel)))
+            out_sc.append([s for s, _ in sel] + [None] * (k - len(sel)))
+    return out_idx, out_sc
+
+
 def e4m3_value(code: int) -> Fraction:
     """Exact value of an OCP E4M3 code (bias 7, 3 mantissa bits, exponent
     field 0 subnormal), written out from the format's definition."""

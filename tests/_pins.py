@@ -258,9 +258,30 @@ def check_sparse_attention(o) -> None:
     assert np.allclose(absw, _sdpa_rows(qa, ka, vabs, idx, batch, scale), rtol=1e-12, atol=1e-13)
 
 
+def check_pivot(o) -> None:
+    """The query-group scan against exact arithmetic on dyadic inputs (groups
+    of 2 and 3, fewer and more candidates than k), and its two special cases:
+    groups of one query with C = k, and C at least T, both equal the exact
+    indexer rows."""
+    for seed, B, S, m, H, D, k, G, C in [(51, 2, 12, 2, 2, 3, 2, 3, 3), (52, 1, 12, 3, 2, 2, 3, 2, 2),
+                                         (53, 2, 8, 1, 2, 2, 2, 4, 5)]:
+        q, w, kc = _dyadic(seed, B, S, m, H, D)
+        rows = np.arange(B * S)
+        bi, bs = brute.topk_pivot(q, w, kc, m, k, G, C)
+        bsf = np.array([[-np.inf if x is None else float(x) for x in r] for r in bs])
+        oi, os_, _ = o.pivot_rows(q, w, kc, m, k, G, C, rows)
+        assert np.array_equal(oi, np.array(bi)) and _same_scores(os_, bsf), ("pivot", seed)
+        ei, es = o.indexer_topk(q, w, kc, m, k)
+        oi, os_, _ = o.pivot_rows(q, w, kc, m, k, 1, k, rows)
+        assert np.array_equal(oi, ei) and _same_scores(os_, es), ("pivot G=1", seed)
+        oi, os_, _ = o.pivot_rows(q, w, kc, m, k, G, S // m, rows)
+        assert np.array_equal(oi, ei) and _same_scores(os_, es), ("pivot C>=T", seed)
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
     check_dyadic_brute_force(o)
     check_fp8_brute_force(o)
     check_decode_brute_force(o)
     check_sparse_attention(o)
+    check_pivot(o)

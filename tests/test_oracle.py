@@ -194,6 +194,10 @@ def test_pins_sparse_attention_library_and_closed_forms():
     _pins.check_sparse_attention(oracle)
 
 
+def test_pins_pivot_brute_force_and_special_cases():
+    _pins.check_pivot(oracle)
+
+
 def test_row_helpers_match_numpy_two_batches():
     """Random bf16 inputs, two batches, rows t < m - 1 included: the max
     |score| over visible keys and the scores of given keys (visible, -1 and

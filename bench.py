@@ -39,6 +39,7 @@ import synth  # noqa: E402
 
 METRIC = "indexer query-key pairs/sec, TFLOPS vs B200 peak, peak HBM GB at 1 GPU"
 METRIC_DECODE = "decode indexer query-key pairs/sec, HBM GB/s vs B200 peak"
+METRIC_PIVOT = "query-group scan: causal pairs/sec of the exact step it stands in for"
 METRIC_LAYER = "sparse attention query-entry pairs/sec, TFLOPS vs B200 peak, indexer share of the layer"
 UNIT = "pairs/s"
 KERNEL_SRC = os.path.join(ROOT, "streaming_top_lightning_b200", "csrc", "k_score_topk.cu")
@@ -713,6 +714,79 @@ def run_decode(args, ds):
     return 0
 
 
+# --------------------------------------------------------------------------- pivot
+
+
+def run_pivot(args, name):
+    """The query-group candidate scan against the exact step on the same
+    inputs: both timed with CUDA events; the recall it gives up is measured
+    by the tests against the oracle."""
+    import torch
+
+    import streaming_top_lightning_b200 as stl
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("pivot workloads run on one GPU")
+    base, G, C = synth.PIVOT_SCANS[name]
+    sh = synth.shape(base)
+    dev = torch.device("cuda", 0)
+    q = synth.gen_q(sh, 0, threads=16)
+    to_bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)  # noqa: E731
+    q_d, kc_d = to_bf(q), to_bf(synth.gen_kc(sh, 0))
+    del q
+    w_d = torch.from_numpy(synth.gen_w(sh, 0)).to(dev)
+    idx = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.int32, device=dev)
+    score = torch.empty((sh.B, sh.S, sh.topk), dtype=torch.float32, device=dev)
+    opts = stl.options()
+    ws_p = torch.empty(stl.pivot_workspace_size(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, G, C, opts),
+                       dtype=torch.uint8, device=dev)
+    ws_e = torch.empty(max(16, stl.workspace_size(sh.B, sh.S, sh.H, sh.D, sh.m, sh.topk, opts)),
+                       dtype=torch.uint8, device=dev)
+
+    def pivot():
+        stl.indexer_pivot(q_d, w_d, kc_d, sh.m, sh.topk, G, C, out=(idx, score), opts=opts,
+                          workspace=ws_p)
+
+    def exact():
+        stl.indexer_topk(q_d, w_d, kc_d, sh.m, sh.topk, out=(idx, score), opts=opts,
+                         workspace=ws_e)
+
+    stream = torch.cuda.current_stream()
+    times = {}
+    for label, fn in (("pivot", pivot), ("exact", exact)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        if stl.device_error() != 0:
+            raise RuntimeError(f"device error during the {label} warm-up")
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(stream)
+        for i in range(args.steps):
+            fn()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        times[label] = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
+    P = causal_pairs(sh.S, sh.T, sh.m) * sh.B
+    ng = sh.S // G
+    reps = (np.arange(ng) * G + G - 1)
+    scan_pairs = int(np.minimum(sh.T, (reps + 1) // sh.m).sum()) * sh.B
+    line = {
+        "metric": METRIC_PIVOT, "value": P / (times["pivot"] / 1e3), "unit": "pairs/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": times["pivot"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; distributions of the workload recipe)",
+        "config": {"workload": name, "indexer": sh.name, "B": sh.B, "S": sh.S, "T": sh.T,
+                   "topk": sh.topk, "group": G, "candidates": C,
+                   "scored_pairs": scan_pairs + sh.B * sh.S * C, "exact_pairs": P},
+        "exact_ms": times["exact"], "speedup_vs_exact": times["exact"] / times["pivot"],
+        "recall": "measured by tests/test_gpu_pivot.py against the oracle",
+        "gpu_launches": args.steps * (stl.decode_plan(sh.B, ng, G - 1, sh.T, sh.H, sh.D, sh.m, C)
+                                      ["launches"] + 3 + 2),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------------- layer
 
 
@@ -813,7 +887,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="long_s256k",
                     choices=sorted(synth.SHAPES) + sorted(synth.DECODE_SHAPES)
-                    + sorted(synth.ATTENTION_LAYERS))
+                    + sorted(synth.ATTENTION_LAYERS) + sorted(synth.PIVOT_SCANS))
     ap.add_argument("--key-chunk", type=int, default=0)
     ap.add_argument("--row-finish", type=int, default=0, choices=(0, 1, 2),
                     help="1: rows finished in the fused kernel; 2: by the merge kernel; "
@@ -828,6 +902,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
+    if args.workload in synth.PIVOT_SCANS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "pivot workloads time the GPU "
+                              "path only; the oracle's scan is timed in the tests"}))
+            return 0
+        return run_pivot(args, args.workload)
     if args.workload in synth.ATTENTION_LAYERS:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "layer workloads time the GPU "

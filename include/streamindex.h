@@ -275,6 +275,32 @@ int si_indexer_decode_workspace_size(int B, int S_q, int t0, int T, int H_I, int
 int si_indexer_decode_plan(int B, int S_q, int t0, int T, int H_I, int d_I, int m, int topk,
                            const si_options* opt, si_plan_info* out);
 
+/* ---- query-group candidate scan ---------------------------------------- */
+
+/*
+ * si_indexer_pivot: an approximate indexer step after the PIVOT news page
+ * (nearby queries select nearly the same keys, so a group of queries shares
+ * one scan).  The queries of each batch form groups of G consecutive
+ * positions.  The group's last position scans every key it can see (the
+ * step of si_indexer_topk for that query) and keeps its C best; each query of
+ * the group then scores only those candidates it can see and keeps its topk
+ * best, in the order and with the padding of si_indexer_topk.  The group's
+ * last query gets its exact row (C >= topk); G = 1 is the exact step, and so
+ * is C >= T.  Work: S/G full scans plus S*C candidate scores.
+ *   Arguments as si_indexer_topk, plus G (S % G == 0) and C (topk <= C <= 2048).
+ *   Workspace: caller-provided, at least si_indexer_pivot_workspace_size
+ *   bytes (the representatives, their candidate rows and the gathered key
+ *   rows: about B*S/G*C*(2*d_I + 12) bytes, plus an indexer workspace).
+ * Errors as si_indexer_topk; SI_ERR_OPTIONS for a bad G or C.
+ */
+int si_indexer_pivot(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                     int d_I, int m, int topk, int G, int C, int32_t* out_idx, float* out_score,
+                     const si_options* opt, void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace si_indexer_pivot needs. */
+int si_indexer_pivot_workspace_size(int B, int S, int H_I, int d_I, int m, int topk, int G, int C,
+                                    const si_options* opt, size_t* bytes);
+
 /* ---- sparse attention over the selected entries -------------------------- */
 
 /*

@@ -196,6 +196,37 @@ def indexer_decode(q, w, kc, t0: int, m: int, topk: int, *, out=None,
     return idx, score
 
 
+def pivot_workspace_size(B: int, S: int, H: int, D: int, m: int, topk: int, G: int, C: int,
+                         opts: SiOptions | None = None) -> int:
+    n = ctypes.c_size_t(0)
+    lib = _lib.load()
+    _lib.check("si_indexer_pivot_workspace_size",
+               lib.si_indexer_pivot_workspace_size(B, S, H, D, m, topk, G, C,
+                                                   ctypes.byref(opts) if opts else None,
+                                                   ctypes.byref(n)))
+    return n.value
+
+
+def indexer_pivot(q, w, kc, m: int, topk: int, G: int, C: int, *, out=None,
+                  opts: SiOptions | None = None, workspace=None, stream=None):
+    """Query-group candidate scan (si_indexer_pivot): groups of G queries share
+    their last query's C best keys as candidates.  Returns (idx, score)."""
+    torch = _torch()
+    _need(q, torch.bfloat16, 4, "q")
+    _need(w, torch.float32, 3, "w")
+    _need(kc, torch.bfloat16, 3, "kc")
+    B, S, H, D = q.shape
+    idx, score = _outputs(B, S, topk, q.device, out)
+    need = pivot_workspace_size(B, S, H, D, m, topk, G, C, opts)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    rc = _lib.load().si_indexer_pivot(_ptr(q), _ptr(w), _ptr(kc), B, S, H, D, m, topk, G, C,
+                                      _ptr(idx), _ptr(score), ctypes.byref(opts) if opts else None,
+                                      _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check("si_indexer_pivot", rc)
+    return idx, score
+
+
 def sparse_attention(qa, ka, va, idx, scale: float | None = None, *, out=None,
                      opts: SiOptions | None = None, stream=None):
     """Multi-query attention of each query's heads over the entries its row of

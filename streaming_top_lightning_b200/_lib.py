@@ -24,7 +24,8 @@ EXPORTS = [
     "si_indexer_topk_fp8", "si_quantize_fp8_rows", "si_topk_scores", "si_status_string",
     "si_get_last_device_error", "si_version", "si_indexer_topk_noalloc", "si_indexer_topk_plan",
     "si_role_cycles", "si_indexer_decode", "si_indexer_decode_workspace_size",
-    "si_indexer_decode_plan", "si_sparse_attention",
+    "si_indexer_decode_plan", "si_sparse_attention", "si_indexer_pivot",
+    "si_indexer_pivot_workspace_size",
 ]
 
 
@@ -93,6 +94,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.si_indexer_decode_plan.argtypes = [I, I, I, I, I, I, I, I, OP,
                                            ctypes.POINTER(SiPlanInfo)]
     lib.si_sparse_attention.argtypes = [P, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, OP, P]
+    lib.si_indexer_pivot.argtypes = [P, P, P, I, I, I, I, I, I, I, I, P, P, OP, P, Z, P]
+    lib.si_indexer_pivot_workspace_size.argtypes = [I, I, I, I, I, I, I, I, OP,
+                                                    ctypes.POINTER(Z)]
     for name in EXPORTS:
         if name != "si_status_string":
             getattr(lib, name).restype = I

@@ -249,6 +249,8 @@ int plan_status(const ScorePlan& sp) {
 struct Problem {
   int B, S, T, t0, m;
   bool decode;
+  int tstride = 1;           // position step between query rows
+  const int* vis = nullptr;  // [B*S] visible keys per row (device), replacing the rule
 };
 
 int check_common(int B, int S, int m, int topk) {
@@ -260,8 +262,8 @@ int check_common(int B, int S, int m, int topk) {
 // Sizes of a prefill (S % m == 0, T = S/m, t0 = 0) or decode call.
 int check_problem(const Problem& pb, int H, int D, int topk) {
   if (pb.decode) {
-    if (pb.B < 1 || pb.S < 1 || pb.T < 1 || pb.t0 < 0 || pb.m < 1 ||
-        (int64_t)pb.t0 + pb.S > 0x7FFFFFFF)
+    if (pb.B < 1 || pb.S < 1 || pb.T < 1 || pb.t0 < 0 || pb.m < 1 || pb.tstride < 1 ||
+        (int64_t)pb.t0 + (int64_t)(pb.S - 1) * pb.tstride + 1 > 0x7FFFFFFF)
       return SI_ERR_DIM;
     if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
   } else {
@@ -294,7 +296,8 @@ int check_indexer(const void* q, const void* w, const void* kc, const Problem& p
 // fixed cost (its query-tile load and its partial list).
 int decode_key_chunk(const Problem& pb, int QT, int sms) {
   const int64_t tiles = (int64_t)pb.B * ((pb.S + QT - 1) / QT);
-  const int vmax = visible_host(pb.t0 + pb.S - 1, pb.T, pb.m);
+  if (pb.vis) return 0;  // per-row counts: tile units, one chunk
+  const int vmax = visible_host(pb.t0 + (pb.S - 1) * pb.tstride, pb.T, pb.m);
   if (vmax <= 128 || tiles >= sms) return 0;
   int best_c = 0;
   int64_t best_cost = -1;
@@ -376,11 +379,12 @@ int run_indexer(bool fp8, const void* q, const float* s_q, const float* w, const
     // a prefill's tiles outnumber the SMs: a unit is a whole tile (loaded
     // once, its chunks in order); a decode step's few tiles are split into
     // (tile, chunk) units that spread over the SMs
-    UnitGrid ug{B, S, T, m, pl.QT, pl.C, g_lo, n_tiles, id_base, pb.decode ? 0 : 1, pb.t0};
+    UnitGrid ug{B,        S,       T,         m,        pl.QT,    pl.C,    g_lo,
+                n_tiles,  id_base, (pb.decode && !pb.vis) ? 0 : 1, pb.t0, pb.tstride, pb.vis};
     ScoreParams p{};
     p.sel = SelParams{B,      S,         T,           m,       K,         pl.QT,
                       sp_plan.CS, sp_plan.cap, pl.L, g_lo, n_tiles, pl.nch_max,
-                      out_idx, out_score, partial, pl.final_rows, pb.t0};
+                      out_idx, out_score, partial, pl.final_rows, pb.t0, pb.tstride, pb.vis};
     p.ug = ug;
     p.w = w;
     p.w_tail = w_tail;
@@ -466,7 +470,7 @@ int noalloc_scratch(void** out) {
 static int host_tile_vmax(const UnitGrid& u, int g) {
   int t = g * u.QT + u.QT - 1;
   if (t > u.S - 1) t = u.S - 1;
-  return visible_host(u.t0 + t, u.T, u.m);
+  return visible_host(u.t0 + t * u.tstride, u.T, u.m);
 }
 
 int host_tile_chunks(const UnitGrid& u, int g) {
@@ -636,10 +640,10 @@ int si_topk_scores(const float* scores, int B, int S, int T, int m, int topk, in
   for (int blk = 0; rc == SI_OK && blk < pl.n_blocks; ++blk) {
     const int g_lo = blk * pl.tb;
     const int n_tiles = pl.G - g_lo < pl.tb ? pl.G - g_lo : pl.tb;
-    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base, 0, 0};
+    UnitGrid ug{B, S, T, m, QT, pl.C, g_lo, n_tiles, id_base, 0, 0, 1, nullptr};
     SelParams sp{B,    S,       T,          m,       topk,    QT,     CS,
                  cap,  pl.L,    g_lo,       n_tiles, pl.nch_max, out_idx, out_score,
-                 partial, pl.final_rows, 0};
+                 partial, pl.final_rows, 0, 1, nullptr};
     const int units = host_count_units(ug);
     int grid = o.grid_ctas > 0 ? o.grid_ctas : dev->sms;
     if (grid > units) grid = units;
@@ -750,6 +754,109 @@ int si_sparse_attention(const void* qa, const void* ka, const void* va, const in
   return launch_sparse_attn(tm_q, p, grid, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SI_OK
              : SI_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ query-group scan
+// Workspace of si_indexer_pivot: the group representatives' q and w, their
+// top-C rows, the sorted candidates, the gathered key rows, the per-query
+// visible counts, then one indexer workspace shared by the two launches.
+struct PivotLayout {
+  size_t qr, wr, ridx, rsc, cand, kcg, vis, iws, total;
+};
+
+static int pivot_layout(const Problem& full, int H, int D, int K, int G, int C,
+                        const si_options* opt, PivotLayout* L, Problem* rep, Problem* rs) {
+  int rc = check_problem(full, H, D, K);
+  if (rc) return rc;
+  if (G < 1 || full.S % G != 0 || C < K || C > SI_MAX_TOPK) return SI_ERR_OPTIONS;
+  const int ng = full.S / G;
+  const int64_t groups = (int64_t)full.B * ng;
+  if (groups * C >= ((int64_t)1 << 31)) return SI_ERR_DIM;
+  *rep = Problem{full.B, ng, full.T, G - 1, full.m, true, G, nullptr};
+  *rs = Problem{(int)groups, G, C, 0, 1, true, 1, nullptr};
+  size_t w1 = 0, w2 = 0;
+  si_options o{};
+  if (opt) o = *opt;
+  o.key_chunk = 0;
+  if ((rc = workspace_for(*rep, H, D, C, &o, &w1))) return rc;
+  if ((rc = workspace_for(*rs, H, D, K, &o, &w2))) return rc;
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t r = at;
+    at += align256(bytes);
+    return r;
+  };
+  L->qr = take((size_t)groups * H * D * 2);
+  L->wr = take((size_t)groups * H * 4);
+  L->ridx = take((size_t)groups * C * 4);
+  L->rsc = take((size_t)groups * C * 4);
+  L->cand = take((size_t)groups * C * 4);
+  L->kcg = take((size_t)groups * C * D * 2);
+  L->vis = take((size_t)full.B * full.S * 4);
+  L->iws = take(std::max(w1, w2));
+  L->total = at;
+  return SI_OK;
+}
+
+int si_indexer_pivot_workspace_size(int B, int S, int H_I, int d_I, int m, int topk, int G, int C,
+                                    const si_options* opt, size_t* bytes) {
+  if (!bytes) return SI_ERR_NULL;
+  PivotLayout L;
+  Problem rep, rs;
+  const int rc = pivot_layout(prefill(B, S, m), H_I, d_I, topk, G, C, opt, &L, &rep, &rs);
+  if (rc == SI_OK) *bytes = L.total;
+  return rc;
+}
+
+int si_indexer_pivot(const void* q, const float* w, const void* kc, int B, int S, int H_I,
+                     int d_I, int m, int topk, int G, int C, int32_t* out_idx, float* out_score,
+                     const si_options* opt, void* workspace, size_t ws_bytes, void* stream) {
+  const Problem full = prefill(B, S, m);
+  int rc = check_indexer(q, w, kc, full, H_I, d_I, topk, out_idx, out_score);
+  if (rc) return rc;
+  PivotLayout L;
+  Problem rep, rs;
+  if ((rc = pivot_layout(full, H_I, d_I, topk, G, C, opt, &L, &rep, &rs))) return rc;
+  if (!workspace || ws_bytes < L.total) return SI_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SI_ERR_ALIGN;
+  DevInfo* dev;
+  if ((rc = dev_info(&dev))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* qr = reinterpret_cast<uint16_t*>(ws + L.qr);
+  float* wr = reinterpret_cast<float*>(ws + L.wr);
+  int32_t* ridx = reinterpret_cast<int32_t*>(ws + L.ridx);
+  float* rsc = reinterpret_cast<float*>(ws + L.rsc);
+  int32_t* cand = reinterpret_cast<int32_t*>(ws + L.cand);
+  uint16_t* kcg = reinterpret_cast<uint16_t*>(ws + L.kcg);
+  int* vis = reinterpret_cast<int*>(ws + L.vis);
+  void* iws = ws + L.iws;
+  const size_t iws_bytes = L.total - L.iws;
+  const PivotParams pp{B, S, S / m, H_I, d_I, m, G, C, S / G};
+  si_options o{};
+  if (opt) o = *opt;
+  o.key_chunk = 0;
+  o.score_event_list = nullptr;
+  o.score_event_count = 0;
+  o.score_events[0] = o.score_events[1] = nullptr;
+  // 1. each group's last query scans its visible keys and keeps C
+  if (launch_pivot_reps(static_cast<const uint16_t*>(q), w, pp, qr, wr, st) != cudaSuccess)
+    return SI_ERR_CUDA;
+  if ((rc = run_indexer(false, qr, nullptr, wr, kc, nullptr, rep, H_I, d_I, C, ridx, rsc, &o, iws,
+                        iws_bytes, st)))
+    return rc;
+  // 2. the candidates sorted by key, their key rows, each query's visible count
+  if (launch_pivot_cands(ridx, static_cast<const uint16_t*>(kc), pp, cand, kcg, vis, st) !=
+      cudaSuccess)
+    return SI_ERR_CUDA;
+  // 3. every query ranks the candidates it sees (q and w viewed as [B*S/G, G, ...])
+  rs.vis = vis;
+  if ((rc = run_indexer(false, q, nullptr, w, kcg, nullptr, rs, H_I, d_I, topk, out_idx,
+                        out_score, &o, iws, iws_bytes, st)))
+    return rc;
+  // 4. candidate positions back to key indices
+  return launch_pivot_remap(out_idx, cand, pp, topk, dev->sms, st) == cudaSuccess ? SI_OK
+                                                                                  : SI_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ decode

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return -1;
         u = UnitInfo{0, 0, 0, 0, 0, 0, 0};
         if (ok) {
-          const int vmax = tile_vmax(p.ug, g);
+          const int vmax = tile_vmax_b(p.ug, b, g);
           u.valid = 1;
           u.b = b;
           u.g = g;

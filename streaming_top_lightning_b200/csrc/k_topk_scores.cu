@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
       named_bar_sync(1, kLoadThreads);
       int b, g, c;
       if (!unit_decode(ug, id, b, g, c)) break;
-      const int vmax = tile_vmax(ug, g);
+      const int vmax = tile_vmax_b(ug, b, g);
       const int kbeg = c * ug.C;
       const int kend = min(kbeg + ug.C, vmax);
       for (int j0 = kbeg;; j0 += CS) {
@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
         for (int qi = 0; qi < QT; ++qi) {
           const int t = g * QT + qi;
           if (t >= sp.S) break;
-          const int lim = min(nk, visible_keys(sp.t0 + t, sp.T, sp.m) - j0);
+          const int lim =
+              min(nk, row_visible(sp.vis, b, sp.S, sp.t0, sp.tstride, t, sp.T, sp.m) - j0);
           const float* src = X + ((int64_t)b * sp.S + t) * sp.T + j0;
           for (int q = tid; q < lim; q += kLoadThreads) st[(size_t)qi * CS + q] = __ldg(src + q);
         }

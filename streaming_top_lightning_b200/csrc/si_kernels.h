@@ -42,6 +42,18 @@ size_t sparse_attn_smem_bytes();
 cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const AttnParams& p, int grid,
                                cudaStream_t stream);
 
+// Sizes of a query-group candidate scan (k_pivot.cu): groups of G queries,
+// ng = S/G per batch, C candidates per group.
+struct PivotParams {
+  int B, S, T, H, D, m, G, C, ng;
+};
+cudaError_t launch_pivot_reps(const uint16_t* q, const float* w, const PivotParams& p,
+                              uint16_t* qr, float* wr, cudaStream_t stream);
+cudaError_t launch_pivot_cands(const int32_t* rep_idx, const uint16_t* kc, const PivotParams& p,
+                               int32_t* cand, uint16_t* kcg, int* vis, cudaStream_t stream);
+cudaError_t launch_pivot_remap(int32_t* out_idx, const int32_t* cand, const PivotParams& p, int K,
+                               int sms, cudaStream_t stream);
+
 // Shared-memory plan of the fused kernel for one problem shape.
 struct ScorePlan {
   int QT;        // queries per tile (nq / H)

@@ -48,6 +48,10 @@ struct SelParams {
   int final_rows;      // 1: every tile is one unit, whose pools are final: the selection
                        // warps write the exact top-K rows themselves (no partial lists)
   int t0;              // sequence position of query row 0 (0 for a whole prefill)
+  int tstride;         // positions of consecutive query rows differ by this (1 but in a
+                       // group-representative scan)
+  const int* vis;      // [B*S] visible keys of each query row, replacing the position
+                       // rule when set (non-decreasing along a batch's rows)
 };
 
 // A unit leaves at most this many candidates per query (a superset of its K
@@ -70,6 +74,13 @@ struct SelSmem {
 SI_DEV int visible_keys(int t, int T, int m) {
   int v = (t + 1) / m;
   return v < T ? v : T;
+}
+
+// Keys query row t of batch b sees: the given count, or min(T, (pos+1)/m) at
+// its position pos = t0 + t*tstride.
+SI_DEV int row_visible(const int* vis, int b, int S, int t0, int tstride, int t, int T, int m) {
+  if (vis) return vis[(int64_t)b * S + t];
+  return visible_keys(t0 + t * tstride, T, m);
 }
 
 __host__ __device__ constexpr int pow2ceil(int x) {
@@ -518,8 +529,9 @@ SI_DEV void select_loop(const SelParams& p, const SelSmem& sm, const Ctl& ctl, i
       if (t >= p.S) continue;
       uint64_t* pool = sm.pool + (size_t)qi * p.cap;
       const long long t_in = role_t0();
-      pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys, visible_keys(p.t0 + t, p.T, p.m),
-                      pool, p.cap, p.K, &sm.npool[qi], &sm.theta[qi], hist, lane, ctl);
+      pool_take_strip(st + (size_t)qi * p.CS, md.j0, md.nkeys,
+                      row_visible(p.vis, md.b, p.S, p.t0, p.tstride, t, p.T, p.m), pool, p.cap,
+                      p.K, &sm.npool[qi], &sm.theta[qi], hist, lane, ctl);
       if (lane == 0) role_add(ctl, R_SEL_INTAKE, t_in);
       if (md.last) {
         const long long t_end = role_t0();
@@ -573,12 +585,23 @@ struct UnitGrid {
                    // order inside it (the tile is loaded once); 0: one unit
                    // per (tile, chunk)
   int t0;          // sequence position of query row 0, the same in every batch
+  int tstride;     // position step between query rows
+  const int* vis;  // per-row visible counts (see SelParams::vis); tile units only
 };
 
+// Visible keys of tile g's last query (the tile's most), by the position rule.
 SI_DEV int tile_vmax(const UnitGrid& u, int g) {
   int t = g * u.QT + u.QT - 1;
   if (t > u.S - 1) t = u.S - 1;
-  return visible_keys(u.t0 + t, u.T, u.m);
+  return visible_keys(u.t0 + t * u.tstride, u.T, u.m);
+}
+
+// The same for batch b, from the per-row counts when given.
+SI_DEV int tile_vmax_b(const UnitGrid& u, int b, int g) {
+  if (!u.vis) return tile_vmax(u, g);
+  int t = g * u.QT + u.QT - 1;
+  if (t > u.S - 1) t = u.S - 1;
+  return u.vis[(int64_t)b * u.S + t];
 }
 
 // Number of chunks of tile g (at least 1, so tiles with no visible key still

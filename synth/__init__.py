@@ -276,6 +276,12 @@ def gen_decode(ds: DecodeShape, seed: int = 0):
 # --------------------------------------------------------------------------- attention
 
 
+# Query-group candidate scans: (indexer workload, group size G, candidates C).
+PIVOT_SCANS = {
+    "pivot_s16k": ("v4flash_s16k", 16, 1024),   # top-512
+    "pivot_s256k": ("long_s256k", 64, 2048),    # top-2048
+}
+
 # A layer: the indexer step of SHAPES[indexer] followed by the attention of
 # 128 heads of dim 128 over the entries it selects.
 ATTENTION_LAYERS = {

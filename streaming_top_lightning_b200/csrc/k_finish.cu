@@ -308,7 +308,11 @@ static FinishShape finish_shape(int K, int L, int nch) {
   return f;
 }
 
-bool finish_takes(int L, int nch) { return (int64_t)L * nch <= kFinishMaxKeys; }
+// One list always; two (a decode step's chunks) when they fit.  More lists go
+// to the merge kernel: a CTA per query costs more than a warp per query once
+// the lists are long and the queries many (S = 32,768, eight chunks of 1,024
+// keys, top-512: 1.8 ms here against 0.4 ms in the merge kernel).
+bool finish_takes(int L, int nch) { return nch <= 2 && (int64_t)L * nch <= kFinishMaxKeys; }
 
 cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,
                                cudaStream_t stream) {

@@ -91,9 +91,9 @@ bool merge_sorts_rows(int K);
 
 // Exact sorted rows from a single candidate list per query (one key chunk);
 // every row comes out sorted, whatever K.
-// The finishing kernel takes a query's lists when they hold at most this many
-// keys together (its shared memory, and the fallback select's byte counters:
-// at most 255 * 32 keys); longer sets go through the merge kernel.
+// The finishing kernel takes a query's one or two lists when they hold at
+// most this many keys together (its shared memory, and the fallback select's
+// byte counters: at most 255 * 32 keys); other sets go through the merge kernel.
 constexpr int kFinishMaxKeys = 8160;
 bool finish_takes(int L, int nch);
 cudaError_t launch_finish_rows(const uint64_t* partial, const SelParams& sp, const UnitGrid& ug,

@@ -159,3 +159,34 @@ def test_plan_hint_options_validated(lib):
         o.plan_heads, o.plan_dim, o.plan_fp8 = heads, dim, fp8
         rc, _ = _ws(lib, 1, 16384, 64, 128, 4, 512, o)
         assert (rc == 0) == ok, (heads, dim, fp8, rc)
+
+
+def test_decode_pivot_attention_argument_errors(lib):
+    """The host-side checks of the decode, query-group and attention entry
+    points (nothing is launched: every case fails before any device access)."""
+    Z = ctypes.c_size_t
+    n = Z(0)
+    # decode: bad position, bad m, bad topk
+    assert lib.si_indexer_decode_workspace_size(1, 1, -1, 16, 64, 128, 4, 8, None,
+                                                ctypes.byref(n)) == -2
+    assert lib.si_indexer_decode_workspace_size(1, 1, 0, 16, 64, 128, 0, 8, None,
+                                                ctypes.byref(n)) == -2
+    assert lib.si_indexer_decode_workspace_size(1, 1, 0, 16, 64, 128, 4, 0, None,
+                                                ctypes.byref(n)) == -3
+    assert lib.si_indexer_decode_workspace_size(1, 2, 9, 16, 64, 128, 4, 8, None,
+                                                ctypes.byref(n)) == 0 and n.value > 0
+    # query-group scan: S not a multiple of G, C below topk, C above 2048
+    for G, C, rc in [(3, 128, -8), (16, 32, -8), (16, 4096, -8), (16, 128, 0)]:
+        assert lib.si_indexer_pivot_workspace_size(1, 512, 64, 128, 4, 64, G, C, None,
+                                                   ctypes.byref(n)) == rc, (G, C)
+    # attention: NULL, heads other than 128, topk, a non-finite scale (fake device
+    # pointers: each call fails before using them)
+    fake = ctypes.c_void_p(256)
+    assert lib.si_sparse_attention(None, fake, fake, fake, 1, 2, 16, 128, 128, 4, 1.0, fake,
+                                   None, None) == -1
+    assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 64, 128, 4, 1.0, fake,
+                                   None, None) == -2
+    assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 0, 1.0, fake,
+                                   None, None) == -3
+    assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 4,
+                                   float("nan"), fake, None, None) == -8

@@ -320,7 +320,8 @@ int si_indexer_pivot_workspace_size(int B, int S, int H_I, int d_I, int m, int t
  * Arithmetic: q.k in fp32 from bf16 products on the tensor cores, softmax
  * in fp32, the probabilities rounded to bf16 for the weighted sum of the
  * value rows (accumulated in fp32).  Limits: 1 <= topk <= 2048; B*S*H_a <
- * 2^31; qa, ka, va, out 16-byte aligned, idx 4-byte aligned; scale finite.
+ * 2^31; qa, ka, va, out 16-byte aligned, idx 4-byte aligned; scale finite and
+ * >= 0 (SI_ERR_OPTIONS otherwise).
  * Options: grid_ctas and timeout_ms are used.  No workspace.
  */
 int si_sparse_attention(const void* qa, const void* ka, const void* va, const int32_t* idx, int B,

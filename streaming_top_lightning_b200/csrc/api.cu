@@ -722,7 +722,7 @@ int si_sparse_attention(const void* qa, const void* ka, const void* va, const in
   if (B < 1 || S < 1 || T < 1 || H_a != 128 || d_a != 128) return SI_ERR_DIM;
   if ((int64_t)B * S * H_a >= ((int64_t)1 << 31)) return SI_ERR_DIM;
   if (topk < 1 || topk > SI_MAX_TOPK) return SI_ERR_TOPK;
-  if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return SI_ERR_OPTIONS;
+  if (!(scale >= 0.0f) || scale == INFINITY) return SI_ERR_OPTIONS;  // NaN fails the first test
   if (!aligned16(qa) || !aligned16(ka) || !aligned16(va) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(idx) & 3u))
     return SI_ERR_ALIGN;

@@ -20,16 +20,19 @@
 //                      thread, 16-byte cp.async into the 128-byte swizzled
 //                      layout; unlisted slots are zero-filled) into one of two
 //                      stages, and load the query's [128 x 128] block by TMA;
-//   MMA warp 8         S = Q K^T (M=128 heads, N=128 entries, K=128) into one
+//   MMA warp 12        S = Q K^T (M=128 heads, N=128 entries, K=128) into one
 //                      of two TMEM score buffers, then O += P V (M=128 heads,
 //                      N=128 dims, K=128 entries) with V read MN-major from
 //                      the same stage, one tile behind, so S of the next tile
 //                      overlaps the softmax of this one;
-//   softmax warps 4-7  one thread per head (its TMEM lane): the running max
-//                      and sum in the log2 domain, P = 2^(s - max) in bf16
-//                      into shared memory (the A operand of P V), the rescale
-//                      of O in TMEM when the max grows, and at the query's end
-//                      O / sum to global memory.
+//   softmax warps 4-11 two per TMEM lane quadrant, so one head per thread in
+//                      each of two warps that split the tile's 128 columns:
+//                      both take the running max over all columns, each the
+//                      exponentials P = 2^(s - max) of its 64 (in bf16, into
+//                      shared memory: the A operand of P V), the rescale of its
+//                      half of O in TMEM when the max grows, its share of the
+//                      row sum (added across the pair at the query's end), and
+//                      O / sum of its half to global memory.
 // Tiles whose 128 slots list no valid entry are skipped; a query that lists
 // none writes zeros.  Every wait is bounded; a CTA that gives up records the
 // error word and leaves.
@@ -41,10 +44,11 @@ namespace {
 constexpr int kAttnH = 128;      // query heads (MMA M)
 constexpr int kAttnD = 128;      // head dim
 constexpr int kAttnTile = 128;   // listed entries per tile (MMA N of Q K^T, K of P V)
-constexpr int kAttnThreads = 288;
+constexpr int kAttnThreads = 416;
 constexpr int kLoadThreads = 128;
-constexpr int kSoftWarp0 = 4;
-constexpr int kMmaWarp = 8;
+constexpr int kSoftWarp0 = 4;   // softmax warps 4-11: two per TMEM lane quadrant
+constexpr int kSoftWarps = 8;
+constexpr int kMmaWarp = 12;
 constexpr uint32_t kTileBytes = kAttnTile * kAttnD * 2;  // 32 KB: one K, V, Q or P block
 constexpr uint32_t kHalf = kTileBytes / 2;               // one 64-column half: [128 x 128 B]
 
@@ -61,6 +65,8 @@ struct AttnCtl {
   uint64_t s_full[2], s_empty[2], p_full, o_done;
   AttnMeta meta[2];
   uint32_t lmask[16][4];  // the loader's masks of the current query's tiles
+  uint64_t xch[4];        // per lane quadrant: the two softmax warps' row sums are in
+  float xsum[2][128];     // [column half][head]: a softmax warp's share of a row's sum
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -156,13 +162,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&cs->kv_full[i]), kLoadThreads);
-      mbar_init(smem_u32(&cs->kv_empty[i]), 5);  // the MMA side and the four softmax warps
+      mbar_init(smem_u32(&cs->kv_empty[i]), 1 + kSoftWarps);  // the MMA side, each softmax warp
       mbar_init(smem_u32(&cs->q_full[i]), 1);
       mbar_init(smem_u32(&cs->q_empty[i]), 1);
       mbar_init(smem_u32(&cs->s_full[i]), 1);
-      mbar_init(smem_u32(&cs->s_empty[i]), 128);
+      mbar_init(smem_u32(&cs->s_empty[i]), kSoftWarps * 32);
     }
-    mbar_init(smem_u32(&cs->p_full), 128);
+    mbar_init(smem_u32(&cs->p_full), kSoftWarps * 32);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&cs->xch[i]), 64);
     mbar_init(smem_u32(&cs->o_done), 1);
     cs->abort = 0u;
     mbar_fence_init();
@@ -333,14 +340,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int st = tid - kSoftWarp0 * 32;  // 0..127: the head, and the TMEM lane
     const int quad = warp & 3;
+    const int st = quad * 32 + lane;          // the head, and the TMEM lane
+    const int half = (warp - kSoftWarp0) >> 2;  // columns [64*half, 64*half + 64) of S, P and O
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t o_col = lane_base + 2 * kAttnTile;
     const float sl2 = p.scale_log2;
     const float ninf = __int_as_float(0xFF800000);
-    uint32_t it = 0, n1 = 0, n2i = 0, n2w = 0;
-    float m = ninf, l = 0.0f;
+    uint32_t it = 0, n1 = 0, n2i = 0, n2w = 0, nx = 0;
+    float m = ninf, l = 0.0f;  // l: this warp's half of the row sum
     bool any = false;  // the current query has had a tile
     for (;;) {
       const int s = (int)(it & 1u);
@@ -361,19 +369,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const uint32_t s_col = lane_base + sb * kAttnTile;
         float v[32];
-        // pass 1: the tile's largest listed score
-        float mx = ninf;
+        // pass 1: the tile's largest listed score (scale >= 0, so the largest
+        // raw dot product scales to the largest logit), four chains, and no
+        // per-slot test on a fully listed group of 32.  Both warps of a lane
+        // quadrant take all 128 columns here, so each has the row maximum
+        // without an exchange; the exponentials below are split by column half.
+        float mx4[4] = {ninf, ninf, ninf, ninf};
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           tmem_ld32(s_col + c * 32, v);
           tmem_ld_wait();
           fence32(v);
           const uint32_t mk = md.mask[c];
+          if (mk == 0xFFFFFFFFu) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if ((mk >> e) & 1u) mx = fmaxf(mx, v[e] * sl2);
+            for (int e = 0; e < 32; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], v[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if ((mk >> e) & 1u) mx4[e & 3] = fmaxf(mx4[e & 3], v[e]);
+          }
         }
-        const float m_new = fmaxf(m, mx);
+        const float mxr = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float m_new = fmaxf(m, mxr * sl2);
         // P and O belong to the previous tile's P V until it completes
         if (n2i > n2w) {
           if (!mbar_wait_warp(smem_u32(&cs->o_done), n2w & 1u, ctl)) break;
@@ -387,7 +405,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float a = m_new > m ? exp2f(m - m_new) : 1.0f;
           l *= a;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 2 * half; c < 2 * half + 2; ++c) {
             tmem_ld32(o_col + c * 32, v);
             tmem_ld_wait();
             fence32(v);
@@ -399,16 +417,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         m = m_new;
         // pass 2: P = 2^(s*scale*log2(e) - m) on listed slots, 0 elsewhere
+        float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
           tmem_ld32(s_col + c * 32, v);
           tmem_ld_wait();
           fence32(v);
           const uint32_t mk = md.mask[c];
+          if (mk == 0xFFFFFFFFu) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            v[e] = ((mk >> e) & 1u) ? exp2f(v[e] * sl2 - m) : 0.0f;
-            l += v[e];
+            for (int e = 0; e < 32; ++e) {
+              v[e] = exp2f(fmaf(v[e], sl2, -m));
+              l4[e & 3] += v[e];
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              v[e] = ((mk >> e) & 1u) ? exp2f(fmaf(v[e], sl2, -m)) : 0.0f;
+              l4[e & 3] += v[e];
+            }
           }
           // entries 32c .. 32c+31 are chunks 4c .. 4c+3 of the head's P row
 #pragma unroll
@@ -424,6 +451,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          : "memory");
           }
         }
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         tc_fence_before();
         mbar_arrive(smem_u32(&cs->s_empty[sb]));
         ++n1;
@@ -435,14 +463,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (md.last) {
         float* orow = p.out + ((int64_t)md.query * kAttnH + st) * kAttnD;
         if (any) {
-          if (!mbar_wait_warp(smem_u32(&cs->o_done), n2w & 1u, ctl)) stop = true;
+          // the row sum: this warp's half plus its partner's (the buffer is
+          // rewritten only after the partner's next P, so once per query is safe)
+          cs->xsum[half][st] = l;
+          mbar_arrive(smem_u32(&cs->xch[quad]));
+          if (!mbar_wait_warp(smem_u32(&cs->xch[quad]), nx & 1u, ctl)) stop = true;
+          ++nx;
+          const float lt = stop ? 1.0f : l + cs->xsum[half ^ 1][st];
+          if (!stop && !mbar_wait_warp(smem_u32(&cs->o_done), n2w & 1u, ctl)) stop = true;
           if (!stop) {
             ++n2w;
             tc_fence_after();
-            const float inv = 1.0f / l;
+            const float inv = 1.0f / lt;
             float v[32];
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * half; c < 2 * half + 2; ++c) {
               tmem_ld32(o_col + c * 32, v);
               tmem_ld_wait();
               fence32(v);
@@ -454,7 +489,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_before();
           }
         } else {
-          for (int c = 0; c < kAttnD; c += 4)
+          for (int c = 64 * half; c < 64 * half + 64; c += 4)
             *reinterpret_cast<float4*>(orow + c) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
       }

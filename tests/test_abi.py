@@ -188,5 +188,6 @@ def test_decode_pivot_attention_argument_errors(lib):
                                    None, None) == -2
     assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 0, 1.0, fake,
                                    None, None) == -3
-    assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 4,
-                                   float("nan"), fake, None, None) == -8
+    for bad in (float("nan"), float("inf"), -0.5):
+        assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 4, bad, fake,
+                                       None, None) == -8

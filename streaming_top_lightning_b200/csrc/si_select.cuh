@@ -307,13 +307,15 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
   const uint32_t lt_mask = (1u << lane) - 1u;
   constexpr int kSteps = 8;
   for (int c0 = 0; c0 < lim; c0 += 64 * kSteps) {
-    const float ninf = __int_as_float(0xFF800000);
+    // slots past the visible keys read as NaN, which compares false with any
+    // threshold (scores are never NaN), so the ballots need no range test
+    const float nan = __int_as_float(0x7FC00000);
     float xa[kSteps], xb[kSteps];
 #pragma unroll
     for (int u = 0; u < kSteps; ++u) {
       const int pa = c0 + 64 * u + lane;
-      xa[u] = pa < lim ? st[pa] : ninf;
-      xb[u] = pa + 32 < lim ? st[pa + 32] : ninf;
+      xa[u] = pa < lim ? st[pa] : nan;
+      xb[u] = pa + 32 < lim ? st[pa + 32] : nan;
     }
     const int nsteps = min(kSteps, (lim - c0 + 63) >> 6);
     int s0 = 0;
@@ -321,9 +323,8 @@ SI_DEV void pool_take_strip(const float* st, int j0, int nkeys, int V, uint64_t*
       uint32_t ma[kSteps], mb[kSteps];
 #pragma unroll
       for (int u = 0; u < kSteps; ++u) {
-        const int pa = c0 + 64 * u + lane;
-        ma[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && pa < lim && xa[u] >= thf);
-        mb[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && pa + 32 < lim && xb[u] >= thf);
+        ma[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && xa[u] >= thf);
+        mb[u] = __ballot_sync(0xFFFFFFFFu, u >= s0 && xb[u] >= thf);
       }
       // the steps [s0, s1) that fit the pool
       int s1 = s0, add = 0;

@@ -894,7 +894,7 @@ def main():
                          "0: the library's choice")
     ap.add_argument("--strip-slots", type=int, default=0, choices=(0, 2, 3, 4),
                     help="score strips in flight between epilogue and selection (0: library's choice)")
-    ap.add_argument("--key-tile", type=int, default=0, choices=(0, 128, 256, 512, 1024),
+    ap.add_argument("--key-tile", type=int, default=0, choices=(0, 32, 64, 128, 256, 512, 1024),
                     help="keys per score strip handed to the selection warps (0: library's choice)")
     ap.add_argument("--topk", type=int, default=0)
     ap.add_argument("--fp8", action="store_true")

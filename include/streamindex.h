@@ -90,11 +90,15 @@ typedef struct si_options {
                            kernel always finishes.  Default 0. */
   int key_tile;         /* keys per score strip handed from the tensor-core
                            epilogue to the selection warps: 128, 256, 512 or
-                           1024 (one to eight 128-key MMA tiles); 0 = the
-                           library's choice.  Default 0. */
+                           1024 (one to eight 128-key MMA tiles), or 32 or 64
+                           (a quarter or half of a tile: each tile's 32-key
+                           lane quadrants are handed over in strips of their
+                           own); 0 = the library's choice.  Default 0. */
   int strip_slots;      /* score strips in flight between the epilogue and
-                           the selection warps: 2 to 4; 0 = the library's
-                           choice.  Default 0. */
+                           the selection warps: 2 to 4, a multiple of
+                           128/key_tile for strips shorter than a tile (4 for
+                           32, 2 or 4 for 64), else SI_ERR_OPTIONS; 0 = the
+                           library's choice.  Default 0. */
   void** score_event_list; /* optional array of score_event_count
                            cudaEvent_t (NULL = none): the call records
                            [2i] on `stream` just before the score-kernel

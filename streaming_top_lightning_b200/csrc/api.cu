@@ -149,9 +149,13 @@ int read_opts(const si_options* o, Opts* out) {
   }
   if (d.key_chunk < 0 || (d.key_chunk % 128) != 0 || d.grid_ctas < 0 || d.scratch_mb > (1 << 20) ||
       d.row_finish < 0 || d.row_finish > 2 ||
-      !(d.key_tile == 0 || d.key_tile == 128 || d.key_tile == 256 || d.key_tile == 512 ||
-        d.key_tile == 1024) ||
+      !(d.key_tile == 0 || d.key_tile == 32 || d.key_tile == 64 || d.key_tile == 128 ||
+        d.key_tile == 256 || d.key_tile == 512 || d.key_tile == 1024) ||
       d.strip_slots < 0 || d.strip_slots == 1 || d.strip_slots > 4 || d.ev_count < 0 ||
+      // strips shorter than a 128-key tile: each tile fills 128/key_tile
+      // strips, each in a slot of its own
+      (d.key_tile == 32 && d.strip_slots != 0 && d.strip_slots != 4) ||
+      (d.key_tile == 64 && d.strip_slots == 3) ||
       !(d.plan_heads == 0 || d.plan_heads == 8 || d.plan_heads == 16 || d.plan_heads == 32 ||
         d.plan_heads == 64) ||
       (d.plan_heads > 0 && !(d.plan_dim == 64 || d.plan_dim == 128)) || d.plan_fp8 < 0 ||

@@ -165,7 +165,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&cs->acc_empty[i]), kEpiThreads);
     }
     for (int i = 0; i < NSL; ++i) {
-      mbar_init(smem_u32(&cs->strip_full[i]), kEpiThreads);
+      // a strip of CS >= 128 keys is written by every epilogue thread; a
+      // shorter one by the two warps (one per column half) of each of its
+      // CS/32 lane quadrants
+      mbar_init(smem_u32(&cs->strip_full[i]), CS >= kM ? kEpiThreads : 2 * CS);
       mbar_init(smem_u32(&cs->strip_empty[i]), kSelWarps * 32);  // every selection lane
     }
     mbar_init(smem_u32(&cs->q_full), 1);
@@ -375,6 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const int cb = ew >> 2;           // column block: queries [cb*QH, cb*QH + QH)
     const int kl = quad * 32 + lane;  // key within the tile
+    // strips shorter than a tile (CS = 32 or 64): a tile fills SUB strips and
+    // this warp's 32 keys belong to strip `sub` of them; its meta is written
+    // by the column-0 warp of the strip's first quadrant
+    const int SUB = CS >= kM ? 1 : kM / CS;
+    const int sub = CS >= kM ? 0 : (quad * 32) / CS;
+    const bool meta_writer = CS >= kM ? ew == 0 : (cb == 0 && quad == sub * (CS / 32));
     uint32_t ring_it = 0, acc_it = 0, strip_it = 0;
     const long long t_role = role_t0();
     for (;;) {
@@ -387,11 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(smem_u32(&cs->unit_empty[r]));
       ++ring_it;
       if (!u.valid) {
-        // no more work: pass the end marker to the selection warps
+        // no more work: pass the end marker to the selection warps (strips
+        // shorter than a tile: through the slot of the tile's first strip,
+        // written by that strip's warps)
         const int slot = (int)(strip_it % (uint32_t)NSL);
-        if (mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u, ctl)) {
-          if (ew == 0 && lane == 0) cs->meta[slot].valid = 0;
-          mbar_arrive(smem_u32(&cs->strip_full[slot]));
+        if (CS >= kM || sub == 0) {
+          if (mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u,
+                             ctl)) {
+            if (meta_writer && lane == 0) cs->meta[slot].valid = 0;
+            mbar_arrive(smem_u32(&cs->strip_full[slot]));
+          }
         }
         break;
       }
@@ -424,10 +438,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int chunk_idx = u.kbeg / sp_chunk;
       bool stop = false;
       for (int i = 0; i < u.ntiles || (i == 0 && u.ntiles == 0); ++i) {
-        const int slot = (int)(strip_it % (uint32_t)NSL);
+        const uint32_t sit = strip_it + (uint32_t)sub;  // this warp's strip
+        const int slot = (int)(sit % (uint32_t)NSL);
         if (pos == 0) {
-          if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((strip_it / NSL) & 1u) ^ 1u,
-                              ctl, R_EPI_WAIT_STRIP)) {
+          if (!mbar_wait_warp(smem_u32(&cs->strip_empty[slot]), ((sit / NSL) & 1u) ^ 1u, ctl,
+                              R_EPI_WAIT_STRIP)) {
             stop = true;
             break;
           }
@@ -476,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j = u.kbeg + i * kM + kl;
             skj = j < sp.T ? p.s_k[(int64_t)u.b * sp.T + j] : 0.0f;
           }
-          float* st = strip + (size_t)slot * QT * CS + (size_t)cb * QH * CS + pos + kl;
+          float* st = strip + (size_t)slot * QT * CS + (size_t)cb * QH * CS + pos + kl - sub * CS;
 #pragma unroll
           for (int ql = 0; ql < QH; ++ql) {
             float s = 0.0f;
@@ -492,8 +507,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jt_end = u.kbeg + (i + 1) * kM;
         const bool last = (i + 1 >= u.ntiles);
         const bool chunk_end = last || jt_end == chunk_next;
-        if (pos >= CS || chunk_end) {
-          if (ew == 0 && lane == 0) {
+        if (CS < kM) {
+          // every tile ends its SUB strips; only the last can end the chunk
+          if (meta_writer && lane == 0) {
+            const int j0 = u.kbeg + i * kM + sub * CS;
+            const int nk = max(0, min(CS, min(chunk_next, u.kend) - j0));
+            cs->meta[slot] = StripMeta{1,  u.b, u.g, chunk_idx, j0, nk,
+                                       (chunk_end && sub == SUB - 1) ? 1 : 0, 0u};
+          }
+          mbar_arrive(smem_u32(&cs->strip_full[slot]));
+          strip_it += (uint32_t)SUB;
+          pos = 0;
+          j_strip = jt_end;
+          if (chunk_end) {
+            chunk_next += sp_chunk;
+            ++chunk_idx;
+          }
+        } else if (pos >= CS || chunk_end) {
+          if (meta_writer && lane == 0) {
             const int nk = max(0, min(CS, min(chunk_next, u.kend) - j_strip));
             cs->meta[slot] =
                 StripMeta{1, u.b, u.g, chunk_idx, j_strip, nk, chunk_end ? 1 : 0, 0u};
@@ -579,7 +610,9 @@ static int strip_max(int QT);
 // key-tile ring slots of one K-block each (kM keys x one swizzle span: a
 // whole key tile when a row fits one span, half of one for bf16 at d_I =
 // 128), a ring of NSL score strips of CS keys per query (cs_req and nsl_req >
-// 0 fix them), the selection pools (cap keys per query), the FP8 weight copy
+// 0 fix them; CS of 32 or 64 keys, a tile's lane quadrants handed over in
+// strips of their own, only when asked for, with NSL a multiple of the
+// tile's 128/CS strips), the selection pools (cap keys per query), the FP8 weight copy
 // and the small control block.  Candidates are ranked lexicographically: a
 // pool of at least 1.5K keys first, then strips of 512 keys, then enough ring
 // slots (below), then a third strip slot, then the larger pool up to 4K keys
@@ -612,10 +645,12 @@ static ScorePlan plan_score_n(bool fp8, int D, int H, int K, int max_smem, int N
   const int min_slots = (NQ == kN ? 2 : 3) * kblocks;
   long best_score[7] = {-1, -1, -1, -1, -1, -1, -1};
   for (int nst = kblocks; nst <= 8; ++nst) {
-    for (int cs = 128; cs <= cs_max; cs <<= 1) {
+    // strips shorter than a tile (32 or 64 keys) only when asked for
+    for (int cs = (cs_req > 0 && cs_req < kM) ? cs_req : kM; cs <= cs_max; cs <<= 1) {
       if (cs_req > 0 && cs != cs_req) continue;
       for (int nsl = 2; nsl <= kMaxSlots; ++nsl) {
         if (nsl_req > 0 && nsl != nsl_req) continue;
+        if (cs < kM && nsl % (kM / cs) != 0) continue;  // a tile's strips: whole slot groups
         const size_t used = fixed + nst * slot_bytes + sizeof(float) * (size_t)nsl * QT * cs;
         if (used + sel_state_bytes(QT, cap_min) > (size_t)max_smem) continue;
         int cap = cap_min;

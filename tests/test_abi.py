@@ -100,8 +100,12 @@ def test_row_finish_option(lib):
 
 
 def test_strip_options_validated(lib):
+    # strips of 32 or 64 keys: a tile's 128/key_tile strips take whole slot groups
     for kt, ss, ok in [(0, 0, True), (128, 2, True), (1024, 4, True), (100, 0, False),
-                       (2048, 0, False), (0, 1, False), (0, 5, False), (256, -1, False)]:
+                       (2048, 0, False), (0, 1, False), (0, 5, False), (256, -1, False),
+                       (32, 0, True), (32, 4, True), (32, 2, False), (32, 3, False),
+                       (64, 0, True), (64, 2, True), (64, 4, True), (64, 3, False),
+                       (16, 0, False), (96, 0, False)]:
         o = _lib.SiOptions(0, 0, 0, 0, 0)
         o.key_tile = kt
         o.strip_slots = ss

@@ -104,7 +104,8 @@ def test_rows_finished_in_fused_kernel_equal_merge(B, S, m, H, D, k):
     _gpu.check_rows(sh, q, w, kc, gi1, gs1, rows)
 
 
-@pytest.mark.parametrize("key_tile,strip_slots", [(128, 2), (256, 3), (512, 4), (1024, 2), (128, 4)])
+@pytest.mark.parametrize("key_tile,strip_slots", [(128, 2), (256, 3), (512, 4), (1024, 2), (128, 4),
+                                                  (32, 4), (64, 2), (64, 4), (32, 0)])
 def test_strip_options_do_not_change_rows(key_tile, strip_slots):
     """The strip length and the number of strips in flight change only how the
     scores travel from the epilogue to the selection warps (and so the pool
@@ -118,6 +119,24 @@ def test_strip_options_do_not_change_rows(key_tile, strip_slots):
     assert torch.equal(gi0, gi1)
     assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
     rows = np.union1d(np.arange(0, sh.S, 31), [sh.S - 1])
+    _gpu.check_rows(sh, q, w, kc, gi1, gs1, rows)
+
+
+@pytest.mark.parametrize("key_tile", [32, 64])
+@pytest.mark.parametrize("B,S,m,chunk", [(2, 1000, 4, 256), (1, 3003, 3, 0), (3, 712, 8, 128)])
+def test_short_strips_ragged(key_tile, B, S, m, chunk):
+    """Strips shorter than a key tile (each lane quadrant of a tile handed
+    over on its own) on ragged shapes, with key chunks that end inside a
+    query tile's reach and units that see no key: the rows equal the default
+    plan's bit for bit and pass the oracle rule."""
+    sh = synth.small(B, S, m, 64, 128, 100, seed=S + key_tile, kc_kind="ar1")
+    q, w, kc = _gpu.inputs(sh, seed=S + key_tile)
+    gi0, gs0 = _gpu.run_bf16(sh, q, w, kc, opts=stl.options(key_chunk=chunk))
+    gi1, gs1 = _gpu.run_bf16(sh, q, w, kc, opts=stl.options(key_chunk=chunk, key_tile=key_tile))
+    assert torch.equal(gi0, gi1)
+    assert torch.equal(gs0.view(torch.int32), gs1.view(torch.int32))
+    _gpu.structural(sh, gi1, gs1, np.arange(B * S))
+    rows = np.union1d(np.arange(0, B * S, 7), [B * S - 1])
     _gpu.check_rows(sh, q, w, kc, gi1, gs1, rows)
 
 

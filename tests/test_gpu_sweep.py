@@ -20,7 +20,7 @@ from tests import _fp8, _gpu
 pytestmark = pytest.mark.gpu
 
 CELLS = ([("key_chunk", c) for c in (1024, 2048, 4096, 8192, 16384)] +
-         [("key_tile", t) for t in (128, 256, 512, 1024)] +
+         [("key_tile", t) for t in (32, 64, 128, 256, 512, 1024)] +
          [("topk", k) for k in (128, 256, 512, 1024, 2048)])
 
 

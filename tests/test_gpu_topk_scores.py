@@ -123,6 +123,24 @@ def test_bit_exact_on_the_indexer_plans(kind, H, D, fp8, k, S, T, m, chunk):
                                   os_.view(np.uint32))
 
 
+@pytest.mark.parametrize("kind", ["normal", "ties"])
+@pytest.mark.parametrize("fp8,k,key_tile", [(0, 512, 32), (0, 512, 64), (1, 2048, 64),
+                                            (0, 2048, 32)])
+def test_bit_exact_on_short_strip_plans(kind, fp8, k, key_tile):
+    """Plans with strips of 32 or 64 keys (a quarter or half of a key tile per
+    hand-over): the selection steps on those strips are bit-exact too."""
+    S, T = 3000, 4096
+    X = synth.gen_scores(1, S, T, seed=k + key_tile, kind=kind)
+    opts = stl.options(plan_heads=64, plan_dim=128, plan_fp8=fp8, key_tile=key_tile)
+    gi, gs = stl.topk_scores(torch.from_numpy(X).cuda(), 1, k, opts=opts)
+    torch.cuda.synchronize()
+    assert stl.device_error() == 0
+    oi, os_ = oracle.topk_scores(X, 1, k)
+    np.testing.assert_array_equal(gi.reshape(-1, k).cpu().numpy(), oi)
+    np.testing.assert_array_equal(gs.reshape(-1, k).cpu().numpy().view(np.uint32),
+                                  os_.view(np.uint32))
+
+
 @pytest.mark.parametrize("H,D,fp8,k", [(64, 128, 0, 512), (64, 128, 0, 2048)])
 def test_increasing_rows_on_the_indexer_plans(H, D, fp8, k):
     """Scores rising along j on the product's plans: every key beats the

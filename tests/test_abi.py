@@ -156,6 +156,23 @@ def test_plan_query(lib):
     assert lib.si_indexer_topk_plan(1, 4096, 64, 128, 4, 64, 0, None, None) == -1
 
 
+def test_plan_short_strips(lib):
+    """Strips of 32 or 64 keys keep the tile and its pools; the strip ring
+    holds whole groups of a tile's 128/key_tile strips (4 for 32; 2 or 4 for
+    64), and the smaller strips leave the pools no less room."""
+    rc, p0 = _plan(lib, 1, 32768, 64, 128, 4, 512)
+    assert rc == 0
+    for kt, ss, want_slots in [(32, 0, 4), (32, 4, 4), (64, 0, 4), (64, 2, 2)]:
+        o = _lib.SiOptions(0, 0, 0, 0, 0)
+        o.key_tile, o.strip_slots = kt, ss
+        for fp8 in (0, 1):
+            rc, p = _plan(lib, 1, 32768, 64, 128, 4, 512, fp8=fp8, opts=o)
+            assert rc == 0, (kt, ss, fp8)
+            assert (p.key_tile, p.strip_slots, p.mma_n) == (kt, want_slots, 256), (kt, ss, fp8)
+            assert p.pool_keys >= p0.pool_keys and p.smem_bytes <= 227 * 1024
+            assert p.launches == p0.launches
+
+
 def test_plan_hint_options_validated(lib):
     for heads, dim, fp8, ok in [(0, 0, 0, True), (64, 128, 0, True), (8, 64, 1, True),
                                 (48, 128, 0, False), (64, 96, 0, False), (64, 128, 2, False)]:

@@ -212,3 +212,43 @@ def test_decode_pivot_attention_argument_errors(lib):
     for bad in (float("nan"), float("inf"), -0.5):
         assert lib.si_sparse_attention(fake, fake, fake, fake, 1, 2, 16, 128, 128, 4, bad, fake,
                                        None, None) == -8
+
+
+# The largest top-k per (fp8, H_I, d_I) that the header documents; every other
+# shape takes top-2048.
+DOCUMENTED_MAX_TOPK = {(0, 8, 128): 1056, (0, 8, 64): 1312, (1, 8, 128): 1280, (1, 8, 64): 1408}
+
+
+@pytest.mark.parametrize("fp8", [0, 1])
+@pytest.mark.parametrize("H", [8, 16, 32, 64])
+@pytest.mark.parametrize("D", [64, 128])
+def test_plan_limits_and_invariants(lib, fp8, H, D):
+    """Host-only planner sweep: the documented largest top-k holds exactly,
+    and every plan below it fits the 227 KB of shared memory, gives each
+    query a pool of at least K + 64 keys, a tile of QT = N / H_I queries, a
+    strip no longer than the tile allows and a strip ring that holds whole
+    groups of a tile's strips."""
+    kmax = DOCUMENTED_MAX_TOPK.get((fp8, H, D), 2048)
+    assert _plan(lib, 1, 16384, H, D, 4, kmax, fp8=fp8)[0] == 0
+    if kmax < 2048:
+        assert _plan(lib, 1, 16384, H, D, 4, kmax + 1, fp8=fp8)[0] == -3
+    for k in sorted({1, 2, 31, 64, 100, 128, 255, 512, 777, 1024, kmax // 2, kmax}):
+        if k > kmax:
+            continue
+        for kt, ss in [(0, 0), (32, 0), (64, 2), (128, 0), (512, 3)]:
+            o = _lib.SiOptions(0, 0, 0, 0, 0)
+            o.key_tile, o.strip_slots = kt, ss
+            rc, p = _plan(lib, 1, 16384, H, D, 4, k, fp8=fp8, opts=o)
+            if rc != 0:
+                # only a strip longer than this tile allows, or pools that no
+                # longer fit beside a requested strip ring, may be refused
+                assert rc in (-8, -3) and kt >= 512, (k, kt, ss, rc)
+                continue
+            assert p.smem_bytes <= 227 * 1024, (k, kt, p.smem_bytes)
+            assert p.pool_keys >= ((k + 64 + 31) // 32) * 32, (k, kt, p.pool_keys)
+            assert p.mma_n in (128, 256) and p.queries_per_tile * H == p.mma_n
+            assert 2 <= p.strip_slots <= 4 and (ss == 0 or p.strip_slots == ss)
+            assert kt == 0 or p.key_tile == kt
+            if p.key_tile < 128:
+                assert p.strip_slots % (128 // p.key_tile) == 0
+            assert p.partial_len >= k and p.partial_len % 32 == 0

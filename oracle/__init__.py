@@ -69,6 +69,12 @@ def declare(lib):
     lib.oracle_indexer_topk_fp8_rows.restype = I
     lib.oracle_score_keys_fp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, I, P]
     lib.oracle_score_keys_fp8_rows.restype = None
+    lib.oracle_mx_scale_byte.argtypes = [ctypes.c_double]
+    lib.oracle_mx_scale_byte.restype = ctypes.c_uint8
+    lib.oracle_quantize_mxfp8_rows.argtypes = [P, L, I, P, P]
+    lib.oracle_quantize_mxfp8_rows.restype = I
+    lib.oracle_indexer_topk_mxfp8_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, P, P]
+    lib.oracle_indexer_topk_mxfp8_rows.restype = I
     lib.oracle_sparse_attention_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double,
                                                  P, P]
     lib.oracle_sparse_attention_rows.restype = I
@@ -347,8 +353,49 @@ def score_keys_fp8_rows(q8_rows, sq_rows, w_rows, k8, s_k, S: int, m: int, rows,
     return out
 
 
+def mx_scale_byte(amax: float, lib=None) -> int:
+    """E8M0 byte of an MX block whose largest magnitude is amax."""
+    return _use(lib).oracle_mx_scale_byte(float(amax))
+
+
+def quantize_mxfp8_rows(x, lib=None):
+    """x [..., cols] uint16 bf16 bits, cols a multiple of 32 -> (codes uint8
+    [..., cols], scale bytes uint8 [..., cols/32]): MX block scaling, one
+    power-of-two scale per 32 consecutive elements."""
+    x = _c(x, np.uint16)
+    shp = x.shape
+    x2 = x.reshape(-1, shp[-1])
+    codes = np.empty(x2.shape, dtype=np.uint8)
+    scales = np.empty((x2.shape[0], max(1, x2.shape[1] // 32)), dtype=np.uint8)
+    if _use(lib).oracle_quantize_mxfp8_rows(_p(x2), x2.shape[0], x2.shape[1], _p(codes),
+                                            _p(scales)) != 0:
+        raise ValueError("oracle_quantize_mxfp8_rows: cols must be a positive multiple of 32")
+    return codes.reshape(shp), scales.reshape(shp[:-1] + (shp[-1] // 32,))
+
+
+def indexer_topk_mxfp8_rows(q8_rows, qs_rows, w_rows, k8, ks, S: int, m: int, k: int, rows,
+                            lib=None):
+    """Oracle top-k of the MXFP8 score (codes and block scales decoded exactly).
+
+    q8_rows [n,H,D] uint8, qs_rows [n,H,D/32] uint8, w_rows [n,H] fp32 for the
+    listed queries; k8 [B,T,D] uint8, ks [B,T,D/32] uint8."""
+    q8_rows, qs_rows = _c(q8_rows, np.uint8), _c(qs_rows, np.uint8)
+    w_rows = _c(w_rows, np.float32)
+    k8, ks, rows = _c(k8, np.uint8), _c(ks, np.uint8), _c(rows, np.int64)
+    n, H, D = q8_rows.shape
+    B = k8.shape[0]
+    idx = np.empty((n, k), dtype=np.int32)
+    sc = np.empty((n, k), dtype=np.float64)
+    rc = _use(lib).oracle_indexer_topk_mxfp8_rows(_p(q8_rows), _p(qs_rows), _p(w_rows), _p(k8),
+              _p(ks), B, S, H, D, m, k, _p(rows), n, _p(idx), _p(sc))
+    if rc != 0:
+        raise ValueError("oracle_indexer_topk_mxfp8_rows: bad arguments")
+    return idx, sc
+
+
 _API = {name: globals()[name] for name in (
     "threads", "visible", "indexer_topk", "indexer_topk_rows", "indexer_topk_rows_absmax",
     "score_keys_rows", "row_absmax_rows", "topk_scores", "e4m3_decode", "e4m3_encode",
     "quantize_e4m3_rows", "indexer_topk_fp8_rows", "score_keys_fp8_rows", "decode_rows",
-    "indexer_decode", "sparse_attention_rows", "pivot_rows")}
+    "indexer_decode", "sparse_attention_rows", "pivot_rows", "mx_scale_byte",
+    "quantize_mxfp8_rows", "indexer_topk_mxfp8_rows")}

@@ -142,3 +142,72 @@ def topk_fp8(q8, s_q, w, k8, s_k, m: int, k: int):
             out_idx.append([j for _, j in sel] + [-1] * (k - len(sel)))
             out_sc.append([s for s, _ in sel] + [None] * (k - len(sel)))
     return out_idx, out_sc
+
+
+def _e4m3_finite_codes():
+    """Non-negative finite E4M3 codes and their exact values, ascending."""
+    return [(c, e4m3_value(c)) for c in range(0x7F)]
+
+
+def mx_quantize_block(bits):
+    """MX block scaling of one block of bf16 values (given as bit patterns),
+    found by search rather than by formula: the scale exponent e is the one
+    integer with 256 <= amax / 2^e < 512 (clamped to [-127, 127]; -127 for a
+    block of zeros), and each element's code is the non-negative E4M3 code
+    whose value is nearest to |x| / 2^e (ties to the even code, 448 for
+    anything above), with x's sign bit.  Returns (codes, scale byte)."""
+    vals = [_bf16(b) for b in bits]
+    amax = max(abs(v) for v in vals)
+    if amax == 0:
+        e = -127
+    else:
+        e = 0
+        while amax / Fraction(2) ** e >= 512:
+            e += 1
+        while amax / Fraction(2) ** e < 256:
+            e -= 1
+        e = max(-127, min(127, e))
+    X = Fraction(2) ** e
+    table = _e4m3_finite_codes()
+    codes = []
+    for b, v in zip(bits, vals):
+        y = abs(v) / X
+        best = None
+        for c, cv in table:
+            d = abs(cv - y)
+            if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+                best = (d, c)
+        codes.append(best[1] | (0x80 if int(b) & 0x8000 else 0))
+    return codes, e + 127
+
+
+def mx_value(code: int, scale_byte: int) -> Fraction:
+    """Exact value of an MX element: its E4M3 value times 2^(byte - 127)."""
+    return e4m3_value(code) * Fraction(2) ** (scale_byte - 127)
+
+
+def topk_mxfp8(q8, qs, w, k8, ks, m: int, k: int):
+    """Exact-rational MXFP8 score top-k; q8 [B,S,H,D], qs [B,S,H,D/32], w
+    [B,S,H], k8 [B,T,D], ks [B,T,D/32]:
+    score = sum_h w * max(0, sum_d mx(q8, qs) * mx(k8, ks)), the block of
+    element d being d // 32."""
+    B, S, H, D = q8.shape
+    T = k8.shape[1]
+    out_idx, out_sc = [], []
+    for b in range(B):
+        for t in range(S):
+            V = visible_count(t, T, m)
+            pairs = []
+            for j in range(V):
+                s = Fraction(0)
+                for h in range(H):
+                    dot = sum((mx_value(int(q8[b, t, h, d]), int(qs[b, t, h, d // 32])) *
+                               mx_value(int(k8[b, j, d]), int(ks[b, j, d // 32]))
+                               for d in range(D)), Fraction(0))
+                    s += _f32(w[b, t, h]) * max(Fraction(0), dot)
+                pairs.append((s, j))
+            pairs.sort(key=lambda p: (-p[0], p[1]))
+            sel = pairs[:k]
+            out_idx.append([j for _, j in sel] + [-1] * (k - len(sel)))
+            out_sc.append([s for s, _ in sel] + [None] * (k - len(sel)))
+    return out_idx, out_sc

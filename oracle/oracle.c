@@ -28,7 +28,8 @@
  *   code  = E4M3 round-to-nearest-even, saturating at 448, of x / scale (fp32)
  * and scored as
  *   score = sum_h w[t,h] * max(0, s_q[t,h]*s_k[j]*sum_d q8[t,h,d]*k8[j,d])
- * with the codes decoded exactly to fp64.
+ * with the codes decoded exactly to fp64.  The MX block-scaled variant (one
+ * power-of-two scale per 32 elements) has its own section below.
  */
 #include <math.h>
 #ifdef _OPENMP
@@ -419,6 +420,121 @@ void oracle_score_keys_fp8_rows(const uint8_t* q8_rows, const float* sq_rows, co
                 k8 + b * T * (int64_t)D, sk + b * T, H, D, j);
         }
     }
+}
+
+/* --------------------------------------------------------------- MX block FP8
+ * Block-scaled E4M3 (MXFP8), from "Microscaling Data Formats for Deep
+ * Learning" (cited in the abstract's reference list) and the OCP MX v1.0
+ * rule it describes: every block of 32 consecutive elements of a row shares
+ * one power-of-two scale X = 2^e, stored as an E8M0 byte e + 127, with
+ *
+ *   e = floor(log2(amax_block)) - 8        (8: the exponent of E4M3's largest
+ *                                           normal value, 448 = 1.75 * 2^8)
+ *
+ * clamped to [-127, 127] (a block of zeros takes -127), and every element
+ * becomes the E4M3 code (round to nearest even, saturating at 448) of x / X.
+ * The scaled block maximum then lies in [256, 512) before rounding.  The
+ * pages give no parameters; the block of 32 and the E4M3 element type are
+ * the MXFP8 format of that specification.  The score is the definition with
+ * every element decoded exactly:
+ *
+ *   score = sum_h w[t,h] * max(0, sum_d q8[t,h,d]*2^eq[t,h,d/32] * k8[j,d]*2^ek[j,d/32])
+ */
+#define MX_BLOCK 32
+
+/* E8M0 byte of a block whose largest magnitude is amax. */
+uint8_t oracle_mx_scale_byte(double amax) {
+    if (!(amax > 0.0)) return 0; /* zeros: e = -127 */
+    int E;
+    (void)frexp(amax, &E); /* amax = f * 2^E, f in [0.5, 1): floor(log2 amax) = E - 1 */
+    int e = (E - 1) - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/* x [rows, cols] bf16 bits, cols a multiple of 32 -> codes [rows, cols] and
+ * scale bytes [rows, cols/32].  Returns -1 on bad sizes. */
+int oracle_quantize_mxfp8_rows(const uint16_t* x, int64_t rows, int cols, uint8_t* codes,
+                               uint8_t* scales) {
+    if (rows < 0 || cols < MX_BLOCK || cols % MX_BLOCK != 0) return -1;
+    int nb = cols / MX_BLOCK;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int blk = 0; blk < nb; blk++) {
+            const uint16_t* xb = x + r * cols + blk * MX_BLOCK;
+            double amax = 0.0;
+            for (int i = 0; i < MX_BLOCK; i++) {
+                double v = fabs(bf16_to_f64(xb[i]));
+                if (v > amax) amax = v;
+            }
+            uint8_t sb = oracle_mx_scale_byte(amax);
+            scales[r * nb + blk] = sb;
+            for (int i = 0; i < MX_BLOCK; i++) {
+                /* x / 2^e is exact in fp64 and in fp32 (8 significant bits,
+                 * far from fp32's range limits at the magnitudes E4M3 keeps) */
+                double y = ldexp(bf16_to_f64(xb[i]), -((int)sb - 127));
+                codes[r * cols + blk * MX_BLOCK + i] = oracle_e4m3_encode((float)y);
+            }
+        }
+    }
+    return 0;
+}
+
+/* MXFP8 score of key j for one query: q8r [H,D] codes, qsr [H,D/32] scale
+ * bytes, wr [H]; k8b [T,D] codes and ksb [T,D/32] scale bytes of its batch. */
+double oracle_score_row_mxfp8(const uint8_t* q8r, const uint8_t* qsr, const float* wr,
+                              const uint8_t* k8b, const uint8_t* ksb, int H, int D, int j) {
+    int nb = D / MX_BLOCK;
+    const uint8_t* kr = k8b + (int64_t)j * D;
+    const uint8_t* ks = ksb + (int64_t)j * nb;
+    double s = 0.0;
+    for (int h = 0; h < H; h++) {
+        double dot = 0.0;
+        for (int d = 0; d < D; d++) {
+            double qv = ldexp(oracle_e4m3_decode(q8r[h * D + d]), (int)qsr[h * nb + d / MX_BLOCK] - 127);
+            double kv = ldexp(oracle_e4m3_decode(kr[d]), (int)ks[d / MX_BLOCK] - 127);
+            dot += qv * kv;
+        }
+        s += (double)wr[h] * (dot > 0.0 ? dot : 0.0);
+    }
+    return s;
+}
+
+/* Top-k of the MXFP8 score for listed queries given by their own rows:
+ * q8_rows [n,H,D], qs_rows [n,H,D/32], w_rows [n,H]; k8 [B,T,D], ks [B,T,D/32].
+ * Same order and padding as oracle_indexer_topk_rows. */
+int oracle_indexer_topk_mxfp8_rows(const uint8_t* q8_rows, const uint8_t* qs_rows,
+                                   const float* w_rows, const uint8_t* k8, const uint8_t* ks,
+                                   int B, int S, int H, int D, int m, int k, const int64_t* rows,
+                                   int n, int32_t* out_idx, double* out_score) {
+    if (B < 1 || S < 1 || H < 1 || D < MX_BLOCK || D % MX_BLOCK != 0 || m < 1 || k < 1 ||
+        S % m != 0)
+        return -1;
+    int T = S / m, nb = D / MX_BLOCK;
+    for (int i = 0; i < n; i++)
+        if (rows[i] < 0 || rows[i] >= (int64_t)B * S) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n; i++) {
+        int64_t b = rows[i] / S;
+        int t = (int)(rows[i] % S);
+        int V = oracle_visible(t, T, m);
+        pair_t* p = (pair_t*)malloc(sizeof(pair_t) * (size_t)(V > 0 ? V : 1));
+        for (int j = 0; j < V; j++) {
+            p[j].s = oracle_score_row_mxfp8(q8_rows + (int64_t)i * H * D,
+                                            qs_rows + (int64_t)i * H * nb, w_rows + (int64_t)i * H,
+                                            k8 + b * T * (int64_t)D, ks + b * T * (int64_t)nb, H,
+                                            D, j);
+            p[j].j = j;
+        }
+        qsort(p, (size_t)V, sizeof(pair_t), cmp_pair);
+        for (int r = 0; r < k; r++) {
+            out_idx[(int64_t)i * k + r] = r < V ? p[r].j : -1;
+            out_score[(int64_t)i * k + r] = r < V ? p[r].s : -INFINITY;
+        }
+        free(p);
+    }
+    return 0;
 }
 
 /* ------------------------------------------------------------ sparse attention

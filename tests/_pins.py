@@ -11,7 +11,8 @@ covers the functions the GPU parity tests and the smoke check call:
 indexer_topk, indexer_topk_rows, indexer_topk_rows_absmax (the rows, their
 scores and the max |score| that scales the tolerance rule), score_keys_rows
 (the score of a key outside the oracle's own top-k), row_absmax_rows and the
-FP8 pair indexer_topk_fp8_rows / score_keys_fp8_rows.
+FP8 pair indexer_topk_fp8_rows / score_keys_fp8_rows, and the MX block
+FP8 functions (mx_scale_byte, quantize_mxfp8_rows, indexer_topk_mxfp8_rows).
 """
 
 from __future__ import annotations
@@ -278,6 +279,96 @@ def check_pivot(o) -> None:
         assert np.array_equal(oi, ei) and _same_scores(os_, es), ("pivot C>=T", seed)
 
 
+def _bf16_bits(x) -> np.ndarray:
+    """fp32 values that bf16 holds exactly -> their bf16 bit patterns."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32)
+    assert np.all((b & 0xFFFF) == 0), "value not exact in bf16"
+    return (b >> 16).astype(np.uint16)
+
+
+def check_mxfp8(o) -> None:
+    """MX block scaling and the MXFP8 score.
+
+    The scale byte at worked values of the rule (the largest magnitude
+    scaled into [256, 512), clamped to 2^-127 .. 2^127, zeros at 2^-127);
+    the quantiser against a search over the E4M3 value table
+    (brute.mx_quantize_block) on blocks of five magnitudes, signed zeros,
+    a saturating block and round-to-even ties; exact round trips of values
+    the format holds; the MXFP8 rows against exact rational arithmetic (two
+    batches, blocks with different scales); and, with one scale per row, the
+    per-row FP8 oracle on the same codes."""
+    # worked values: amax -> e = floor(log2 amax) - 8, byte e + 127
+    for amax, byte in [(1.0, 119), (448.0, 127), (500.0, 127), (511.0, 127), (256.0, 127),
+                       (255.0, 126), (512.0, 128), (0.0, 0), (3 * 2.0 ** -130, 0),
+                       (2.0 ** -118, 1), (2.0 ** 135, 254), (2.0 ** 140, 254), (0.75, 118)]:
+        assert o.mx_scale_byte(amax) == byte, ("mx scale byte", amax)
+    # the quantiser against the search, block by block
+    g = np.random.default_rng(41)
+    blocks = []
+    for mag in (1e-30, 1e-3, 1.0, 7.0, 1e20):
+        blocks.append(g.standard_normal(32) * mag)
+    blocks.append(np.zeros(32))
+    sat = g.standard_normal(32)
+    sat[5] = 500.0  # e = 0: 500 saturates to 448; -3 and 1.0625 (a tie) keep theirs
+    sat[6], sat[7], sat[8] = -3.0, 1.0625, -0.0
+    blocks.append(sat)
+    tiny = g.standard_normal(32) * 1e-39  # bf16 subnormals: the scale clamps at 2^-127
+    blocks.append(tiny)
+    x = np.stack(blocks).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16).reshape(4, 64)  # truncation: any bf16
+    codes, scales = o.quantize_mxfp8_rows(bits)
+    assert codes.shape == (4, 64) and scales.shape == (4, 2)
+    for r in range(4):
+        for blk in range(2):
+            bc, bs = brute.mx_quantize_block(bits[r, blk * 32:(blk + 1) * 32].tolist())
+            assert scales[r, blk] == bs, ("mx scale", r, blk)
+            assert codes[r, blk * 32:(blk + 1) * 32].tolist() == bc, ("mx codes", r, blk)
+    # exact round trip: E4M3 values times 2^e whose block maximum fixes e
+    vals = np.array([brute.e4m3_value(c) for c in range(0x7F)], dtype=object)
+    for e in (-20, 0, 9):
+        pick = g.choice(np.arange(0x7F), size=32)
+        pick[0] = 0x7E  # 448: the block's maximum, so its exponent is e
+        v = np.array([float(vals[c]) * 2.0 ** e for c in pick], dtype=np.float32)
+        v[1::2] *= -1
+        c2, s2 = o.quantize_mxfp8_rows(_bf16_bits(v).reshape(1, 32))
+        assert s2[0, 0] == e + 127
+        back = np.array([float(brute.mx_value(int(c), int(s2[0, 0]))) for c in c2[0]])
+        assert np.array_equal(back, v.astype(np.float64)), ("mx round trip", e)
+    # MXFP8 rows against exact rational arithmetic
+    B, S, m, H, D, k = 2, 6, 2, 2, 64, 3
+    T = S // m
+    fin = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    q8 = g.choice(fin, size=(B, S, H, D))
+    k8 = g.choice(fin, size=(B, T, D))
+    qs = g.integers(118, 136, size=(B, S, H, D // 32)).astype(np.uint8)
+    ks = g.integers(118, 136, size=(B, T, D // 32)).astype(np.uint8)
+    w = (g.integers(-8, 9, size=(B, S, H)) / 8).astype(np.float32)
+    bi, bsc = brute.topk_mxfp8(q8, qs, w, k8, ks, m, k)
+    rows = np.arange(B * S)
+    oi, os_ = o.indexer_topk_mxfp8_rows(q8.reshape(B * S, H, D), qs.reshape(B * S, H, D // 32),
+                                        w.reshape(B * S, H), k8, ks, S, m, k, rows)
+    assert np.array_equal(oi, np.array(bi)), ("mxfp8 rows", oi, bi)
+    for r in range(B * S):
+        for c in range(k):
+            want = -np.inf if bsc[r][c] is None else float(bsc[r][c])
+            assert os_[r, c] == want or abs(os_[r, c] - want) <= 1e-14 * abs(want), ("mx score",
+                                                                                   r, c)
+    # one scale per row: the per-row FP8 oracle with s = 2^(byte - 127)
+    qb = g.integers(118, 136, size=(B, S, H)).astype(np.uint8)
+    kb = g.integers(118, 136, size=(B, T)).astype(np.uint8)
+    qs1 = np.repeat(qb[..., None], D // 32, axis=-1)
+    ks1 = np.repeat(kb[..., None], D // 32, axis=-1)
+    mi, ms = o.indexer_topk_mxfp8_rows(q8.reshape(B * S, H, D), qs1.reshape(B * S, H, D // 32),
+                                       w.reshape(B * S, H), k8, ks1, S, m, k, rows)
+    fi, fs = o.indexer_topk_fp8_rows(q8.reshape(B * S, H, D),
+                                     np.ldexp(1.0, qb.astype(np.int32) - 127).astype(
+                                         np.float32).reshape(B * S, H),
+                                     w.reshape(B * S, H), k8,
+                                     np.ldexp(1.0, kb.astype(np.int32) - 127).astype(np.float32),
+                                     S, m, k, rows)
+    assert np.array_equal(mi, fi) and np.allclose(ms, fs, rtol=1e-13, atol=0), "mx vs fp8"
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
     check_dyadic_brute_force(o)
@@ -285,3 +376,4 @@ def run_all(o) -> None:
     check_decode_brute_force(o)
     check_sparse_attention(o)
     check_pivot(o)
+    check_mxfp8(o)

@@ -225,3 +225,7 @@ def test_row_helpers_match_numpy_two_batches():
     assert np.all(np.isnan(got[~vis]))
     np.testing.assert_allclose(got[vis], s[np.repeat(rows, 40).reshape(-1, 40)[vis], js[vis]],
                                rtol=1e-12, atol=1e-15)
+
+
+def test_pins_mxfp8():
+    _pins.check_mxfp8(oracle)

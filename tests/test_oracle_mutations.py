@@ -92,6 +92,18 @@ MUTATIONS = {
     "attn_normaliser_skips_first": ("            double Z = 0.0;\n            for (int r = 0; r < k; r++) {",
                                     "            double Z = 0.0;\n            for (int r = 1; r < k; r++) {"),
     "attn_absw_without_abs": ("                    ah[d] += p * fabs(v);", "                    ah[d] += p * v;"),
+    # MX block FP8: the scale rule, the quantiser and the score
+    "mx_exponent_off_by_one": ("    int e = (E - 1) - 8;", "    int e = (E - 1) - 7;"),
+    "mx_round_instead_of_floor": ("    int e = (E - 1) - 8;", "    int e = E - 8;"),
+    "mx_no_low_clamp": ("    if (e < -127) e = -127;\n", ""),
+    "mx_zero_block_scale_one": ("if (!(amax > 0.0)) return 0;", "if (!(amax > 0.0)) return 127;"),
+    "mx_signed_block_max": ("double v = fabs(bf16_to_f64(xb[i]));", "double v = bf16_to_f64(xb[i]);"),
+    "mx_key_scale_of_block_0": ("(int)ks[d / MX_BLOCK] - 127", "(int)ks[0] - 127"),
+    "mx_query_scales_of_head_0": ("(int)qsr[h * nb + d / MX_BLOCK] - 127",
+                                  "(int)qsr[d / MX_BLOCK] - 127"),
+    "mx_no_relu": ("        s += (double)wr[h] * (dot > 0.0 ? dot : 0.0);",
+                   "        s += (double)wr[h] * dot;"),
+    "mx_no_batch_offset": ("k8 + b * T * (int64_t)D, ks + b * T * (int64_t)nb", "k8, ks"),
 }
 
 

@@ -369,8 +369,29 @@ def check_mxfp8(o) -> None:
     assert np.array_equal(mi, fi) and np.allclose(ms, fs, rtol=1e-13, atol=0), "mx vs fp8"
 
 
+def check_topk_scores(o) -> None:
+    """The selection on given fp32 values (the bit-exact tests' reference)
+    against numpy's lexsort with -0 folded into +0, on normal, tied,
+    constant and infinite scores, with fewer visible keys than k."""
+    for kind in ["normal", "ties", "const", "inf"]:
+        X = synth.gen_scores(2, 40, 13, seed=3, kind=kind)
+        for m, k in [(3, 4), (1, 13), (2, 20)]:
+            oi, os_ = o.topk_scores(X, m, k)
+            for r in range(2 * 40):
+                b, t = divmod(r, 40)
+                V = min(13, (t + 1) // m)
+                x = X[b, t, :V].copy()
+                key = np.where(x == 0, np.float32(0), x)  # -0 -> +0
+                order = np.lexsort((np.arange(V), -key.astype(np.float64)))[:k]
+                n = order.size
+                assert np.array_equal(oi[r, :n], order), ("topk_scores order", kind, r)
+                assert np.array_equal(os_[r, :n].view(np.uint32), x[order].view(np.uint32))
+                assert np.all(oi[r, n:] == -1) and np.all(np.isneginf(os_[r, n:])), "padding"
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
+    check_topk_scores(o)
     check_dyadic_brute_force(o)
     check_fp8_brute_force(o)
     check_decode_brute_force(o)

@@ -104,6 +104,18 @@ MUTATIONS = {
     "mx_no_relu": ("        s += (double)wr[h] * (dot > 0.0 ? dot : 0.0);",
                    "        s += (double)wr[h] * dot;"),
     "mx_no_batch_offset": ("k8 + b * T * (int64_t)D, ks + b * T * (int64_t)nb", "k8, ks"),
+    # topk_scores: the selection on given fp32 values
+    "topk_scores_tie_reversed": (
+        "    const pairf_t* y = (const pairf_t*)b;\n    if (x->s > y->s) return -1;\n"
+        "    if (x->s < y->s) return 1;\n    return (x->j < y->j) ? -1 : (x->j > y->j);",
+        "    const pairf_t* y = (const pairf_t*)b;\n    if (x->s > y->s) return -1;\n"
+        "    if (x->s < y->s) return 1;\n    return (x->j > y->j) ? -1 : (x->j < y->j);"),
+    "topk_scores_pad_zero": ("                out_score[(int64_t)i * k + r] = -INFINITY;",
+                             "                out_score[(int64_t)i * k + r] = 0.0f;"),
+    "topk_scores_visibility_all_T": ("        const float* xr = X + row * (int64_t)T;\n"
+                                     "        pairf_t* p = (pairf_t*)malloc(sizeof(pairf_t) * (size_t)(V > 0 ? V : 1));",
+                                     "        const float* xr = X + row * (int64_t)T;\n        V = T;\n"
+                                     "        pairf_t* p = (pairf_t*)malloc(sizeof(pairf_t) * (size_t)(V > 0 ? V : 1));"),
 }
 
 

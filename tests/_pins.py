@@ -389,9 +389,42 @@ def check_topk_scores(o) -> None:
                 assert np.all(oi[r, n:] == -1) and np.all(np.isneginf(os_[r, n:])), "padding"
 
 
+def check_fp8_quantiser(o) -> None:
+    """The per-row E4M3 quantiser: the encoder against torch's float8_e4m3fn
+    conversion (a library route) on values spread over the format's range,
+    including the subnormal grid and exact ties, and hand values from the
+    format's definition (saturation, signed zero); the row scale is the
+    row's largest magnitude over 448, which lands that element on +-448."""
+    import torch
+
+    g = np.random.default_rng(5)
+    ys = (np.exp2(g.uniform(-11, 8.8, size=4000)) * g.choice([-1, 1], size=4000)).astype(np.float32)
+    ties = np.array([1.0625, 1.1875, 3 * 2.0 ** -10, 5 * 2.0 ** -10, 2.0 ** -11, 17.0, 19.0, 464.0],
+                    dtype=np.float32)
+    ys = np.concatenate([ys[np.abs(ys) <= 448], ties])
+    want = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([o.e4m3_encode(float(y)) for y in ys], dtype=np.uint8)
+    assert np.array_equal(got, want), "e4m3 encoder vs torch"
+    assert o.e4m3_encode(500.0) == 0x7E and o.e4m3_encode(-1000.0) == 0xFE, "saturation"
+    assert o.e4m3_encode(-0.0) == 0x80 and o.e4m3_encode(0.0) == 0x00, "signed zero"
+    sh = synth.small(1, 16, 4, 4, 64, 8, seed=2)
+    q = synth.gen_q(sh, 2)
+    codes, scale = o.quantize_e4m3_rows(q)
+    x = synth.bf16_bits_to_f32(q)
+    amax = np.abs(x).max(axis=-1)
+    assert np.array_equal(scale, (amax / np.float32(448)).astype(np.float32)), "row scale"
+    am = np.abs(x).argmax(axis=-1)
+    top = np.take_along_axis(codes, am[..., None], axis=-1)[..., 0]
+    assert np.all((top & 0x7F) == 0x7E), "row maximum on 448"
+    y = (x / scale[..., None]).astype(np.float32)
+    want = torch.from_numpy(np.clip(y, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, want), "row codes vs torch"
+
+
 def run_all(o) -> None:
     check_hand_cases(o)
     check_topk_scores(o)
+    check_fp8_quantiser(o)
     check_dyadic_brute_force(o)
     check_fp8_brute_force(o)
     check_decode_brute_force(o)

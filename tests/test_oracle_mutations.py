@@ -116,6 +116,13 @@ MUTATIONS = {
                                      "        pairf_t* p = (pairf_t*)malloc(sizeof(pairf_t) * (size_t)(V > 0 ? V : 1));",
                                      "        const float* xr = X + row * (int64_t)T;\n        V = T;\n"
                                      "        pairf_t* p = (pairf_t*)malloc(sizeof(pairf_t) * (size_t)(V > 0 ? V : 1));"),
+    # the per-row E4M3 quantiser
+    "e4m3_ties_away": ("    return fmod(f, 2.0) == 0.0 ? f : f + 1.0;", "    return f + 1.0;"),
+    "e4m3_saturate_to_nan": ("    if (a >= 448.0) return sign | 0x7E;", "    if (a >= 448.0) return sign | 0x7F;"),
+    "e4m3_drop_sign": ("    uint8_t sign = signbit(y) ? 0x80 : 0x00;", "    uint8_t sign = 0x00;"),
+    "e4m3_row_scale_240": ("        volatile float s = amax / 448.0f;", "        volatile float s = amax / 240.0f;"),
+    "e4m3_row_amax_signed": ("            float v = fabsf((float)bf16_to_f64(xr[c]));",
+                             "            float v = (float)bf16_to_f64(xr[c]);"),
 }
 
 

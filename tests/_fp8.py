@@ -65,7 +65,9 @@ def fp8_oracle_ref(sh, w, q8r, sqr, k8, sk, rows, k):
 
 def quant_error_bound(sh, q, w, kc, q8r, sqr, k8, sk, rows, js):
     """E(j) of the module docstring for keys js[i, :] of the listed rows
-    (nan where js < 0)."""
+    (nan where js < 0); q8r and sqr hold the codes and scales of exactly
+    those rows, in the same order."""
+    assert len(q8r) == len(rows) == len(sqr) == len(js)
     tab = e4m3_table()
     qf = synth.bf16_bits_to_f32(q.reshape(-1, sh.H, sh.D)[rows]).astype(np.float64)
     qh = tab[q8r] * sqr.astype(np.float64)[..., None]
@@ -111,7 +113,8 @@ def accuracy_vs_bf16(sh, q, w, kc, q8r, sqr, k8, sk, rows, gi_rows, bf16_ref, to
         missed = np.setdiff1d(o, g)
         assert missed.size >= 1, rows[i]
         js = np.concatenate([extra, missed]).astype(np.int32)[None, :]
-        E = quant_error_bound(sh, q, w, kc, q8r, sqr, k8, sk, rows[i:i + 1], js)[0]
+        E = quant_error_bound(sh, q, w, kc, q8r[i:i + 1], sqr[i:i + 1], k8, sk, rows[i:i + 1],
+                              js)[0]
         s = oracle.score_keys_rows(qr[i:i + 1], wr[i:i + 1], kc, sh.S, sh.m, rows[i:i + 1], js)[0]
         ne = extra.size
         floor = np.max(s[ne:] - E[ne:]) - 2 * tol_rel * amax[i]

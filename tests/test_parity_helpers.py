@@ -76,3 +76,26 @@ def test_structural_catches_order_and_padding():
     bad[rs, 1] = 0
     with pytest.raises(AssertionError):
         _gpu.structural(sh, bad, sc, rows)
+
+
+def test_decode_check_on_oracle_rows():
+    """The decode tests' check (check_decode) with the decode oracle's rows as
+    the device's: they pass; the rows of the sequences in the wrong order,
+    or one query's row given to its neighbour, fail."""
+    from tests.test_gpu_decode import _decode_shape, check_decode
+
+    ds = _decode_shape(3, 4, 700, 300, 8, 64, 3, 16, seed=5)
+    q, w, kc = synth.gen_decode(ds, seed=5)
+    oi, os_, _ = oracle.indexer_decode(q, w, kc, ds.t0, ds.seq.m, ds.seq.topk)
+    gi, gs = oi.astype(np.int32), os_.astype(np.float32)
+    check_decode(ds, q, w, kc, gi, gs)
+    check_decode(ds, q, w, kc, gi, gs, batches=[2, 0])
+    S_q = ds.S_q
+    swapped = np.concatenate([gi[S_q:2 * S_q], gi[:S_q], gi[2 * S_q:]])
+    sws = np.concatenate([gs[S_q:2 * S_q], gs[:S_q], gs[2 * S_q:]])
+    with pytest.raises(AssertionError):
+        check_decode(ds, q, w, kc, swapped, sws)
+    shifted, shs = gi.copy(), gs.copy()
+    shifted[1], shs[1] = gi[0], gs[0]
+    with pytest.raises(AssertionError):
+        check_decode(ds, q, w, kc, shifted, shs)

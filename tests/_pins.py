@@ -133,6 +133,11 @@ def check_fp8_brute_force(o) -> None:
     oi, os_ = o.indexer_topk_fp8_rows(q8.reshape(B * S, H, D), s_q.reshape(B * S, H),
                                       w.reshape(B * S, H), k8, s_k, S, m, k, rows)
     assert np.array_equal(oi, np.array(bi)), ("fp8 rows", oi, bi)
+    # a reversed row subset with its own rows' codes: each row finds its batch
+    sub = rows[::-1][::2].copy()
+    si, ss = o.indexer_topk_fp8_rows(q8.reshape(B * S, H, D)[sub], s_q.reshape(B * S, H)[sub],
+                                     w.reshape(B * S, H)[sub], k8, s_k, S, m, k, sub)
+    assert np.array_equal(si, oi[sub]) and np.array_equal(ss, os_[sub]), "fp8 row subset"
     for r in range(B * S):
         for c in range(k):
             want = -np.inf if bs[r][c] is None else float(bs[r][c])
@@ -272,6 +277,10 @@ def check_pivot(o) -> None:
         bsf = np.array([[-np.inf if x is None else float(x) for x in r] for r in bs])
         oi, os_, _ = o.pivot_rows(q, w, kc, m, k, G, C, rows)
         assert np.array_equal(oi, np.array(bi)) and _same_scores(os_, bsf), ("pivot", seed)
+        # a subset of the rows in another order gives those rows' results
+        sub = rows[::-1][::2].copy()
+        si, ss, _ = o.pivot_rows(q, w, kc, m, k, G, C, sub)
+        assert np.array_equal(si, oi[sub]) and _same_scores(ss, os_[sub]), ("pivot rows", seed)
         ei, es = o.indexer_topk(q, w, kc, m, k)
         oi, os_, _ = o.pivot_rows(q, w, kc, m, k, 1, k, rows)
         assert np.array_equal(oi, ei) and _same_scores(os_, es), ("pivot G=1", seed)
